@@ -1,0 +1,410 @@
+"""Plain, slow reference model of Tensor Core MMA arithmetic (the oracle).
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module;
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may use it.  It shares no code with the CUDA kernels.
+
+What it computes: one output element of a 16x16x16 tile MMA, D = C + A.B,
+under the "characterise-then-simulate" arithmetic models recovered in
+
+  "Hawkeye: Reproducing GPU-Level Non-Determinism (MLSys 2026)" (reading notes),
+   - Key observations, Obs. 1: the (2^11-1)^2 product survives exactly
+     inside the dot-product path;
+   - Key observations, Obs. 2: Ampere FP16 accumulates in two stages,
+     {C, P[1..8]} then the result with P[9..16]; Hopper sums all 16
+     products and C in a single 17-term stage;
+   - Key observations, Obs. 3: internal significand of 24 bits (Ampere) or
+     25 bits (Hopper) including the implicit bit; alignment shifts round
+     toward zero (truncation); products are not normalised before
+     accumulation; subnormal products are not renormalised; the write-back
+     to the output precision also rounds toward zero;
+   - Recovered Ampere FP16 pipeline (Algorithms 12-14, Figure 1): products
+     kept at extended precision ("m_raw << 3"), pyramid GroupSum with
+     truncating alignment "m_i >> delta_e", toward-zero write-back; Hopper
+     difference; BF16 extended range with a final cast to FP32 (overflow to
+     infinity) and the max-exponent threshold of -133;
+   - Experiments and results, Algorithm 10: BF16 intermediates may exceed
+     the FP32 finite range as long as the final value is back in range,
+     otherwise the result saturates to infinity;
+   - Key observations, Obs. 4: large MatMuls are compositions of the
+     16x16 tiles.
+
+and the xorsum fingerprint of
+  "How AEGIS Turns Training Redundancy into Evidence" (AEGIS, chapter 6),
+   section "Redundancy already exists in the training computation".
+
+Everything is done with Python integers, so no step can round by accident.
+Where the pages leave a point open, the reading taken is stated next to the
+code (readings R1..R12, listed with the same numbers in the design notes).
+
+Conventions
+-----------
+* A decoded finite value is (s, e, m): value = (-1)^s * m * 2^(e - p), with
+  e = max(field, 1) - bias and m = frac + (field != 0) * 2^p.  Subnormals keep
+  e = 1 - bias and have no implicit bit (Obs. 3, "subnormal products are not
+  renormalised").
+* A *term* is (s, e, A) with A >= 0 an integer holding F fraction bits below
+  2^e: value = (-1)^s * A * 2^(e - F).  A product of two decoded values is
+  the term (sa ^ sb, ea + eb, ma * mb * 2^(F - 2p)), i.e. the exact product
+  with no normalisation; for FP16 under the Ampere model F - 2p = 3, which is
+  the "m_raw << 3" of the recovered pipeline (reading R1).
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Iterable, Optional, Sequence
+
+# ---------------------------------------------------------------------------
+# Formats
+# ---------------------------------------------------------------------------
+
+
+@dataclass(frozen=True)
+class Fmt:
+    """A binary floating-point storage format.
+
+    ieee_specials=True: an all-ones exponent field is Inf (frac 0) or NaN.
+    ieee_specials=False: the OCP E4M3 convention, no infinities, and only the
+    all-ones exponent with all-ones fraction is NaN.
+    """
+
+    name: str
+    ebits: int
+    p: int  # stored fraction bits
+    bias: int
+    ieee_specials: bool = True
+
+    @property
+    def nbits(self) -> int:
+        return 1 + self.ebits + self.p
+
+    @property
+    def emin(self) -> int:  # exponent of the smallest normal
+        return 1 - self.bias
+
+    @property
+    def emax(self) -> int:  # exponent of the largest finite binade
+        top = (1 << self.ebits) - 1
+        return (top - 1 if self.ieee_specials else top) - self.bias
+
+
+FP16 = Fmt("fp16", 5, 10, 15)
+BF16 = Fmt("bf16", 8, 7, 127)
+E4M3 = Fmt("e4m3", 4, 3, 7, ieee_specials=False)
+FP32 = Fmt("fp32", 8, 23, 127)
+
+FORMATS = {"fp16": FP16, "bf16": BF16, "e4m3": E4M3}
+
+CANONICAL_NAN32 = 0x7FC00000  # reading R9: every NaN result is this pattern
+
+
+@dataclass(frozen=True)
+class Val:
+    kind: str  # "fin", "inf" or "nan"
+    s: int
+    e: int = 0
+    m: int = 0
+
+    @property
+    def is_zero(self) -> bool:
+        return self.kind == "fin" and self.m == 0
+
+
+def decode(fmt: Fmt, bits: int) -> Val:
+    """Split a bit pattern into (sign, unbiased exponent, integer significand).
+
+    Subnormals take the minimum exponent and no implicit bit; this is the
+    representation that enters the products unchanged (Obs. 3; target-test
+    table row "Subnormal Behavior Detection").
+    """
+    bits &= (1 << fmt.nbits) - 1
+    s = bits >> (fmt.ebits + fmt.p)
+    field = (bits >> fmt.p) & ((1 << fmt.ebits) - 1)
+    frac = bits & ((1 << fmt.p) - 1)
+    top = (1 << fmt.ebits) - 1
+    if fmt.ieee_specials and field == top:
+        return Val("nan" if frac else "inf", s)
+    if not fmt.ieee_specials and field == top and frac == (1 << fmt.p) - 1:
+        return Val("nan", s)
+    e = max(field, 1) - fmt.bias
+    m = frac + ((1 << fmt.p) if field != 0 else 0)
+    return Val("fin", s, e, m)
+
+
+# ---------------------------------------------------------------------------
+# Models
+# ---------------------------------------------------------------------------
+
+
+@dataclass(frozen=True)
+class Model:
+    """An accumulation model.
+
+    F       fraction bits kept below 2^e_max when a group is aligned; the
+            internal significand is W = F + 1 bits including the implicit bit
+            (24 for Ampere, 25 for Hopper: Obs. 3 / target-test table row
+            "Internal Precision Detection").
+    groups  product indices of each accumulation stage, in order.  The first
+            stage also holds C; every later stage also holds the normalised
+            result of the stage before it (Obs. 2).
+    e_floor lower bound applied to each group's max exponent (reading R7 of
+            "the max-exponent threshold of -133"), or None for no bound.
+    """
+
+    name: str
+    F: int
+    groups: tuple
+    e_floor: Optional[int] = -133
+
+    @property
+    def W(self) -> int:
+        return self.F + 1
+
+    @property
+    def k(self) -> int:
+        return sum(len(g) for g in self.groups)
+
+
+AMPERE = Model("ampere", 23, (tuple(range(0, 8)), tuple(range(8, 16))))
+HOPPER = Model("hopper", 24, (tuple(range(0, 16)),))
+MODELS = {"ampere": AMPERE, "hopper": HOPPER}
+
+# Which (model, format) pairs exist.  FP8 E4M3 is characterised on Hopper
+# only (Obs. 3, "possible failure cases"); Ampere has no FP8 MMA (reading R11).
+SUPPORTED = {("ampere", "fp16"), ("ampere", "bf16"), ("hopper", "fp16"),
+             ("hopper", "bf16"), ("hopper", "e4m3")}
+
+
+# ---------------------------------------------------------------------------
+# Terms and groups
+# ---------------------------------------------------------------------------
+
+
+@dataclass(frozen=True)
+class Term:
+    s: int
+    e: int
+    A: int  # >= 0, F fraction bits below 2^e
+
+
+def product_term(model: Model, fmt: Fmt, a: Val, b: Val) -> Term:
+    """Exact, unnormalised product (Obs. 1 and Obs. 3; "m_raw << 3").
+
+    The significand product ma*mb has 2p fraction bits and may lie in
+    [1, 4) (or below 1 for subnormal factors); it is only rescaled to F
+    fraction bits, never rounded and never renormalised.
+    """
+    shift = model.F - 2 * fmt.p
+    assert shift >= 0, "model grid must be at least as fine as an exact product"
+    return Term(a.s ^ b.s, a.e + b.e, (a.m * b.m) << shift)
+
+
+def c_term(model: Model, cfmt: Fmt, c: Val) -> Term:
+    """The accumulator input C as a term of the first group (reading R8:
+    an fp32 C, subnormal or not, enters like any decoded value)."""
+    shift = model.F - cfmt.p
+    assert shift >= 0
+    return Term(c.s, c.e, c.m << shift)
+
+
+@dataclass(frozen=True)
+class GroupResult:
+    S: int  # signed integer sum
+    e_max: int  # the group's alignment exponent; value = S * 2^(e_max - F)
+
+
+def group_sum(model: Model, terms: Iterable[Term]) -> Optional[GroupResult]:
+    """GroupSum: align every term to the group's largest exponent and add.
+
+    * only nonzero terms take part in the max (reading R5);
+    * e_max is raised to the model's floor when it is lower (reading R7);
+    * each term is shifted right by e_max - e_i on its MAGNITUDE, dropping
+      the low bits, i.e. truncation toward zero ("m_i >> delta_e, truncated
+      rather than IEEE nearest-even", recovered pipeline; target-test table
+      row "Rounding Mode Detection"); the sign is applied afterwards;
+    * the aligned integers are added exactly, so the order inside a group
+      does not matter.
+    Returns None when every term is zero.
+    """
+    nz = [t for t in terms if t.A != 0]
+    if not nz:
+        return None
+    e_max = max(t.e for t in nz)
+    if model.e_floor is not None:
+        e_max = max(e_max, model.e_floor)
+    S = 0
+    for t in nz:
+        T = t.A >> (e_max - t.e)  # e_max >= t.e, so this is a right shift
+        S += -T if t.s else T
+    return GroupResult(S, e_max)
+
+
+def normalise(model: Model, g: GroupResult) -> Optional[Term]:
+    """Turn a nonzero stage result into a term of W significant bits.
+
+    The excess low bits are truncated (toward zero, like every other
+    rounding step of the model; reading R4).  The exponent is unbounded:
+    BF16 intermediates may exceed the FP32 range (Algorithm 10).
+    Returns None when the stage summed to exactly zero, which then
+    contributes no term to the next stage.
+    """
+    if g.S == 0:
+        return None
+    mag = abs(g.S)
+    L = mag.bit_length()
+    W = model.W
+    if L > W:
+        M, e1 = mag >> (L - W), g.e_max + (L - W)
+    else:
+        M, e1 = mag << (W - L), g.e_max - (W - L)
+    return Term(1 if g.S < 0 else 0, e1, M)
+
+
+# ---------------------------------------------------------------------------
+# Final write-back
+# ---------------------------------------------------------------------------
+
+
+def encode_inf(out: Fmt, s: int) -> int:
+    return (s << (out.nbits - 1)) | (((1 << out.ebits) - 1) << out.p)
+
+
+def cast_rz(model: Model, g: GroupResult, out: Fmt = FP32) -> int:
+    """Write the final sum back to ``out`` rounding toward zero.
+
+    Value V = |S| * 2^(e_max - F), E = floor(log2 V).
+      E >  out.emax  -> infinity of the sum's sign (Algorithm 10);
+      E >= out.emin  -> normal, significand truncated to p+1 bits;
+      otherwise      -> gradual underflow, truncated to the subnormal grid
+                        (reading R9); a result that truncates to nothing is a
+                        zero carrying the sign of S.
+    A zero S is handled by the caller (zero-sign rule).
+    """
+    assert g.S != 0 and out.ieee_specials
+    s = 1 if g.S < 0 else 0
+    mag = abs(g.S)
+    E = g.e_max - model.F + mag.bit_length() - 1
+    sign_bit = s << (out.nbits - 1)
+    if E > out.emax:
+        return encode_inf(out, s)
+    if E >= out.emin:
+        # significand with implicit bit: floor(V / 2^(E - p))
+        sh = (g.e_max - model.F) - (E - out.p)
+        sig = mag << sh if sh >= 0 else mag >> (-sh)
+        assert (1 << out.p) <= sig < (2 << out.p)
+        return sign_bit | ((E + out.bias) << out.p) | (sig - (1 << out.p))
+    # subnormal grid 2^(emin - p)
+    sh = (g.e_max - model.F) - (out.emin - out.p)
+    q = mag << sh if sh >= 0 else mag >> (-sh)
+    assert q < (1 << out.p)
+    return sign_bit | q
+
+
+# ---------------------------------------------------------------------------
+# One output element
+# ---------------------------------------------------------------------------
+
+
+def mma_element(model: Model, fmt: Fmt, a_bits: Sequence[int], b_bits: Sequence[int],
+                c_bits: int, cfmt: Fmt = FP32, out: Fmt = FP32) -> int:
+    """D[m][n] = C[m][n] + sum_k A[m][k] * B[k][n] under ``model``.
+
+    ``a_bits`` is row m of the A tile, ``b_bits`` column n of the B tile
+    (k = 0..K-1; the pages' P[i] is k = i - 1, reading R10), ``c_bits`` the
+    accumulator input.  Returns the bit pattern of D[m][n] in ``out``.
+    """
+    K = model.k
+    assert len(a_bits) == K and len(b_bits) == K
+    a = [decode(fmt, x) for x in a_bits]
+    b = [decode(fmt, x) for x in b_bits]
+    c = decode(cfmt, c_bits)
+
+    # Special values (reading R9; the pages say nothing about NaN or Inf
+    # operands): any NaN operand, or Inf times zero, gives the canonical NaN;
+    # otherwise infinite terms decide the result, and Inf of both signs is
+    # NaN.
+    if c.kind == "nan" or any(v.kind == "nan" for v in a + b):
+        return _nan(out)
+    inf_signs = set()
+    if c.kind == "inf":
+        inf_signs.add(c.s)
+    for ak, bk in zip(a, b):
+        if ak.kind == "inf" or bk.kind == "inf":
+            if ak.is_zero or bk.is_zero:
+                return _nan(out)
+            inf_signs.add(ak.s ^ bk.s)
+    if len(inf_signs) == 2:
+        return _nan(out)
+    if inf_signs:
+        return encode_inf(out, inf_signs.pop())
+
+    P = [product_term(model, fmt, a[k], b[k]) for k in range(K)]
+    carry: Optional[Term] = c_term(model, cfmt, c)
+    result: Optional[GroupResult] = None
+    for gi, idx in enumerate(model.groups):
+        terms = ([carry] if carry is not None else []) + [P[k] for k in idx]
+        result = group_sum(model, terms)
+        if gi + 1 < len(model.groups):
+            carry = normalise(model, result) if result is not None else None
+
+    if result is None or result.S == 0:
+        # Zero-sign rule (reading R12): the IEEE toward-zero sum of zeros is
+        # -0 only when every addend is -0; any cancellation gives +0.
+        all_neg_zero = c.is_zero and c.s == 1 and all(
+            (a[k].is_zero or b[k].is_zero) and (a[k].s ^ b[k].s) == 1 for k in range(K))
+        return (1 << (out.nbits - 1)) if all_neg_zero else 0
+    return cast_rz(model, result, out)
+
+
+def _nan(out: Fmt) -> int:
+    if out is FP32:
+        return CANONICAL_NAN32
+    return (((1 << out.ebits) - 1) << out.p) | (1 << (out.p - 1))
+
+
+# ---------------------------------------------------------------------------
+# Tiles, GEMM, fingerprints
+# ---------------------------------------------------------------------------
+
+
+def mma_tile(model: Model, fmt: Fmt, A, B, C) -> list:
+    """One 16x16x16 tile: A[m][k], B[k][n] in ``fmt``; C[m][n] fp32 bits."""
+    K = model.k
+    return [[mma_element(model, fmt, A[m], [B[k][n] for k in range(K)], C[m][n])
+             for n in range(len(B[0]))] for m in range(len(A))]
+
+
+def gemm_element(model: Model, fmt: Fmt, A, B, c_bits: int, m: int, n: int) -> int:
+    """One element of a large MatMul composed of 16x16x16 tiles.
+
+    K is walked in 16-wide chunks in ascending order and each chunk's fp32
+    result is the next chunk's C (Obs. 4: a large MatMul is a deterministic
+    composition of tiles; the chunk order is the one this library fixes).
+    """
+    K = len(A[m])
+    assert K % 16 == 0
+    d = c_bits
+    for j in range(0, K, 16):
+        d = mma_element(model, fmt, A[m][j:j + 16], [B[k][n] for k in range(j, j + 16)], d)
+    return d
+
+
+def gemm(model: Model, fmt: Fmt, A, B, C) -> list:
+    M, N = len(A), len(B[0])
+    return [[gemm_element(model, fmt, A, B, C[m][n], m, n) for n in range(N)] for m in range(M)]
+
+
+def xorsum(words: Iterable[int]) -> int:
+    """The AEGIS xorsum: the XOR of a tensor's 32-bit words (reading R6)."""
+    r = 0
+    for w in words:
+        r ^= w & 0xFFFFFFFF
+    return r
+
+
+def tile_fingerprints(D) -> list:
+    """xorsum of every 16x16 tile of D, tiles in row-major tile-grid order."""
+    M, N = len(D), len(D[0])
+    return [xorsum(D[m][n] for m in range(i, i + 16) for n in range(j, j + 16))
+            for i in range(0, M, 16) for j in range(0, N, 16)]

@@ -1,0 +1,370 @@
+/*
+ * Plain C restatement of the Tensor Core MMA arithmetic model (the oracle).
+ *
+ * TEST INFRASTRUCTURE ONLY: loaded by tests/, __graft_entry__.smoke() and the
+ * CPU-baseline leg of bench.py.  It shares no code, header or table with the
+ * CUDA library; both are written from the same description:
+ *
+ *   "Hawkeye: Reproducing GPU-Level Non-Determinism (MLSys 2026)" reading
+ *   notes -- Key observations Obs. 1-4; the target-test table; the recovered
+ *   Ampere FP16 pipeline (Algorithms 12-14, Figure 1) with its Hopper and BF16
+ *   paragraphs; Experiments and results, Algorithm 10.
+ *   "How AEGIS Turns Training Redundancy into Evidence", section "Redundancy
+ *   already exists in the training computation" (xorsum fingerprint).
+ *
+ * One output element is computed at a time, exactly as the Python oracle in
+ * mma_model.py does it, with 64-bit integers (every aligned term is below
+ * 2^26 and every group sum below 2^31, so nothing can overflow).  Threads only
+ * split independent output elements between them.
+ *
+ * Readings of points the pages leave open carry the same numbers (R1..R12)
+ * as in mma_model.py.
+ */
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORC_AMPERE = 0, ORC_HOPPER = 1 };
+enum { ORC_FP16 = 0, ORC_BF16 = 1, ORC_E4M3 = 2 };
+
+#define ORC_NAN 0x7FC00000u
+#define E_FLOOR (-133) /* reading R7: floor on each group's max exponent */
+
+typedef struct {
+  int kind; /* 0 finite, 1 inf, 2 nan */
+  int s, e;
+  int64_t m;
+} val_t;
+
+typedef struct {
+  int ebits, p, bias, ieee;
+} fmt_t;
+
+static const fmt_t FMT_IN[3] = {{5, 10, 15, 1}, {8, 7, 127, 1}, {4, 3, 7, 0}};
+static const fmt_t FMT_F32 = {8, 23, 127, 1};
+
+/* Decode: e = max(field,1) - bias, m = frac (+ 2^p when field != 0).
+ * Subnormals are not renormalised (Obs. 3). */
+static val_t decode(const fmt_t *f, uint32_t bits) {
+  val_t v;
+  uint32_t top = (1u << f->ebits) - 1u;
+  uint32_t field = (bits >> f->p) & top;
+  uint32_t frac = bits & ((1u << f->p) - 1u);
+  v.s = (int)((bits >> (f->p + f->ebits)) & 1u);
+  v.e = 0;
+  v.m = 0;
+  if (f->ieee && field == top) {
+    v.kind = frac ? 2 : 1;
+    return v;
+  }
+  if (!f->ieee && field == top && frac == (1u << f->p) - 1u) {
+    v.kind = 2;
+    return v;
+  }
+  v.kind = 0;
+  v.e = (int)(field ? field : 1) - f->bias;
+  v.m = (int64_t)frac + (field ? ((int64_t)1 << f->p) : 0);
+  return v;
+}
+
+typedef struct {
+  int s, e;
+  int64_t A; /* magnitude, F fraction bits below 2^e */
+} term_t;
+
+typedef struct {
+  int F;           /* 23 Ampere, 24 Hopper (internal width F+1) */
+  int ngroups;     /* 2 Ampere, 1 Hopper */
+  int gbeg[2], gend[2];
+} model_t;
+
+static void get_model(int model, model_t *md) {
+  if (model == ORC_AMPERE) {
+    md->F = 23;
+    md->ngroups = 2;
+    md->gbeg[0] = 0; md->gend[0] = 8;   /* {C, P[1..8]} */
+    md->gbeg[1] = 8; md->gend[1] = 16;  /* {stage-1 result, P[9..16]} */
+  } else {
+    md->F = 24;
+    md->ngroups = 1;
+    md->gbeg[0] = 0; md->gend[0] = 16;  /* {C, P[1..16]} */
+    md->gbeg[1] = 16; md->gend[1] = 16;
+  }
+}
+
+/* GroupSum: max exponent over the nonzero terms (R5), raised to the floor
+ * (R7); every magnitude is shifted right by e_max - e_i, dropping the low
+ * bits (toward zero), then signed and added exactly.  Returns 0 when every
+ * term is zero, else 1 with *S and *emax set. */
+static int group_sum(const term_t *t, int n, int64_t *S, int *emax) {
+  int i, any = 0, em = 0;
+  int64_t sum = 0;
+  for (i = 0; i < n; i++) {
+    if (t[i].A == 0) continue;
+    if (!any || t[i].e > em) em = t[i].e;
+    any = 1;
+  }
+  if (!any) return 0;
+  if (em < E_FLOOR) em = E_FLOOR;
+  for (i = 0; i < n; i++) {
+    int d;
+    int64_t T;
+    if (t[i].A == 0) continue;
+    d = em - t[i].e; /* >= 0 */
+    T = d >= 62 ? 0 : (t[i].A >> d);
+    sum += t[i].s ? -T : T;
+  }
+  *S = sum;
+  *emax = em;
+  return 1;
+}
+
+static int bitlen64(uint64_t x) {
+  int n = 0;
+  while (x) { n++; x >>= 1; }
+  return n;
+}
+
+/* Final write-back to fp32, rounding toward zero; overflow gives infinity
+ * (Algorithm 10); below 2^-126 the value is truncated onto the subnormal grid
+ * (R9). S must be nonzero. */
+static uint32_t cast_fp32_rz(int F, int64_t S, int emax) {
+  uint32_t sign = S < 0 ? 0x80000000u : 0u;
+  uint64_t mag = (uint64_t)(S < 0 ? -S : S);
+  int L = bitlen64(mag);
+  int E = emax - F + L - 1;
+  int sh;
+  uint64_t q;
+  if (E > 127) return sign | 0x7F800000u;
+  if (E >= -126) {
+    sh = (emax - F) - (E - 23); /* significand = floor(V / 2^(E-23)) */
+    q = sh >= 0 ? (mag << sh) : (mag >> (-sh));
+    return sign | ((uint32_t)(E + 127) << 23) | (uint32_t)(q - (1u << 23));
+  }
+  sh = (emax - F) - (-149); /* subnormal grid 2^-149 */
+  if (sh >= 0) q = mag << sh;
+  else q = (-sh) >= 64 ? 0 : (mag >> (-sh));
+  return sign | (uint32_t)q;
+}
+
+static uint32_t load_in(int fmt, const void *p, size_t idx) {
+  if (fmt == ORC_E4M3) return ((const uint8_t *)p)[idx];
+  return ((const uint16_t *)p)[idx];
+}
+
+/* One element of D = C + A.B over a 16-long k range.  a(k) = A[a_off +
+ * k*a_step], b(k) = B[b_off + k*b_step]. */
+static uint32_t mma_element(int model, int fmt, const void *Ap, size_t a_off, size_t a_step,
+                            const void *Bp, size_t b_off, size_t b_step, uint32_t cbits) {
+  const fmt_t *f = &FMT_IN[fmt];
+  model_t md;
+  val_t a[16], b[16], c;
+  term_t P[16], terms[17];
+  int k, g, n, have_carry, any_inf = 0, inf_sign = 0;
+  term_t carry;
+  int64_t S = 0;
+  int emax = 0, have_result = 0;
+
+  get_model(model, &md);
+  for (k = 0; k < 16; k++) {
+    a[k] = decode(f, load_in(fmt, Ap, a_off + (size_t)k * a_step));
+    b[k] = decode(f, load_in(fmt, Bp, b_off + (size_t)k * b_step));
+  }
+  c = decode(&FMT_F32, cbits);
+
+  /* Special values (R9): NaN anywhere, or Inf x 0, gives NaN; infinities of
+   * one sign give that infinity; both signs give NaN. */
+  if (c.kind == 2) return ORC_NAN;
+  for (k = 0; k < 16; k++)
+    if (a[k].kind == 2 || b[k].kind == 2) return ORC_NAN;
+  if (c.kind == 1) { any_inf = 1; inf_sign = c.s; }
+  for (k = 0; k < 16; k++) {
+    if (a[k].kind == 1 || b[k].kind == 1) {
+      int s = a[k].s ^ b[k].s;
+      if ((a[k].kind == 0 && a[k].m == 0) || (b[k].kind == 0 && b[k].m == 0)) return ORC_NAN;
+      if (any_inf && s != inf_sign) return ORC_NAN;
+      any_inf = 1;
+      inf_sign = s;
+    }
+  }
+  if (any_inf) return (inf_sign ? 0x80000000u : 0u) | 0x7F800000u;
+
+  /* Exact unnormalised products at F fraction bits (Obs. 1, Obs. 3). */
+  for (k = 0; k < 16; k++) {
+    P[k].s = a[k].s ^ b[k].s;
+    P[k].e = a[k].e + b[k].e;
+    P[k].A = (a[k].m * b[k].m) << (md.F - 2 * f->p);
+  }
+  carry.s = c.s;
+  carry.e = c.e;
+  carry.A = c.m << (md.F - 23);
+  have_carry = 1;
+
+  for (g = 0; g < md.ngroups; g++) {
+    n = 0;
+    if (have_carry) terms[n++] = carry;
+    for (k = md.gbeg[g]; k < md.gend[g]; k++) terms[n++] = P[k];
+    have_result = group_sum(terms, n, &S, &emax);
+    if (g + 1 < md.ngroups) {
+      /* Stage result normalised to W = F+1 bits, truncated (R4); a stage
+       * that sums to exactly zero contributes no term. */
+      have_carry = 0;
+      if (have_result && S != 0) {
+        uint64_t mag = (uint64_t)(S < 0 ? -S : S);
+        int L = bitlen64(mag), W = md.F + 1;
+        carry.s = S < 0;
+        if (L > W) { carry.A = (int64_t)(mag >> (L - W)); carry.e = emax + (L - W); }
+        else { carry.A = (int64_t)(mag << (W - L)); carry.e = emax - (W - L); }
+        have_carry = 1;
+      }
+    }
+  }
+
+  if (!have_result || S == 0) {
+    /* Zero-sign rule (R12): -0 only if C and every product are -0. */
+    int all_neg = (c.m == 0 && c.s == 1);
+    for (k = 0; k < 16 && all_neg; k++)
+      if (!((a[k].m == 0 || b[k].m == 0) && (a[k].s ^ b[k].s) == 1)) all_neg = 0;
+    return all_neg ? 0x80000000u : 0u;
+  }
+  return cast_fp32_rz(md.F, S, emax);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Exported entry points                                                    */
+/* ------------------------------------------------------------------------ */
+
+int orc_supported(int model, int fmt) {
+  if (model != ORC_AMPERE && model != ORC_HOPPER) return 0;
+  if (fmt < ORC_FP16 || fmt > ORC_E4M3) return 0;
+  if (model == ORC_AMPERE && fmt == ORC_E4M3) return 0; /* R11 */
+  return 1;
+}
+
+uint32_t orc_mma_element(int model, int fmt, const void *a16, const void *b16, uint32_t c) {
+  return mma_element(model, fmt, a16, 0, 1, b16, 0, 1, c);
+}
+
+/* Tiles: A, B [ntiles][16][16] (A is (m,k), B is (k,n)); C, D [ntiles][16][16]
+ * fp32 bit patterns; C may be NULL (all +0). */
+typedef struct {
+  int model, fmt;
+  const void *A, *B;
+  const uint32_t *C;
+  uint32_t *D;
+  size_t begin, end;
+} tiles_job_t;
+
+static void *tiles_worker(void *arg) {
+  tiles_job_t *j = (tiles_job_t *)arg;
+  size_t t;
+  int m, n;
+  for (t = j->begin; t < j->end; t++)
+    for (m = 0; m < 16; m++)
+      for (n = 0; n < 16; n++) {
+        size_t o = t * 256 + (size_t)m * 16 + n;
+        j->D[o] = mma_element(j->model, j->fmt, j->A, t * 256 + (size_t)m * 16, 1, j->B,
+                              t * 256 + (size_t)n, 16, j->C ? j->C[o] : 0u);
+      }
+  return NULL;
+}
+
+int orc_tiles(int model, int fmt, const void *A, const void *B, const uint32_t *C, uint32_t *D,
+              size_t ntiles, int nthreads) {
+  pthread_t th[256];
+  tiles_job_t jobs[256];
+  int i;
+  if (!orc_supported(model, fmt)) return -1;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  for (i = 0; i < nthreads; i++) {
+    jobs[i].model = model; jobs[i].fmt = fmt; jobs[i].A = A; jobs[i].B = B;
+    jobs[i].C = C; jobs[i].D = D;
+    jobs[i].begin = ntiles * (size_t)i / (size_t)nthreads;
+    jobs[i].end = ntiles * (size_t)(i + 1) / (size_t)nthreads;
+    pthread_create(&th[i], NULL, tiles_worker, &jobs[i]);
+  }
+  for (i = 0; i < nthreads; i++) pthread_join(th[i], NULL);
+  return 0;
+}
+
+/* GEMM: A [M][K], B [K][N], C, D [M][N] (fp32 bits, C may be NULL), row-major.
+ * K is walked in 16-wide chunks in ascending order; each chunk's result is
+ * the next chunk's C (Obs. 4 composition, fixed chunk order).  Only the
+ * output rows [row_begin, row_end) and columns [col_begin, col_end) are
+ * computed. */
+uint32_t orc_gemm_element(int model, int fmt, int M, int N, int K, const void *A, const void *B,
+                          const uint32_t *C, int m, int n) {
+  uint32_t d = C ? C[(size_t)m * N + n] : 0u;
+  int j;
+  (void)M;
+  for (j = 0; j < K; j += 16)
+    d = mma_element(model, fmt, A, (size_t)m * K + j, 1, B, (size_t)j * N + n, (size_t)N, d);
+  return d;
+}
+
+typedef struct {
+  int model, fmt, M, N, K;
+  const void *A, *B;
+  const uint32_t *C;
+  uint32_t *D;
+  int col_begin, col_end;
+  int next_row, row_end;
+  pthread_mutex_t *mu;
+} gemm_job_t;
+
+static void *gemm_worker(void *arg) {
+  gemm_job_t *j = (gemm_job_t *)arg;
+  for (;;) {
+    int m, n;
+    pthread_mutex_lock(j->mu);
+    m = j->next_row < j->row_end ? j->next_row++ : -1;
+    pthread_mutex_unlock(j->mu);
+    if (m < 0) break;
+    for (n = j->col_begin; n < j->col_end; n++)
+      j->D[(size_t)m * j->N + n] = orc_gemm_element(j->model, j->fmt, j->M, j->N, j->K, j->A, j->B, j->C, m, n);
+  }
+  return NULL;
+}
+
+int orc_gemm_region(int model, int fmt, int M, int N, int K, const void *A, const void *B,
+                    const uint32_t *C, uint32_t *D, int row_begin, int row_end, int col_begin,
+                    int col_end, int nthreads) {
+  pthread_t th[256];
+  pthread_mutex_t mu = PTHREAD_MUTEX_INITIALIZER;
+  gemm_job_t job;
+  int i;
+  if (!orc_supported(model, fmt)) return -1;
+  if (M % 16 || N % 16 || K % 16 || M <= 0 || N <= 0 || K <= 0) return -1;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  job.model = model; job.fmt = fmt; job.M = M; job.N = N; job.K = K;
+  job.A = A; job.B = B; job.C = C; job.D = D;
+  job.col_begin = col_begin; job.col_end = col_end;
+  job.next_row = row_begin; job.row_end = row_end; job.mu = &mu;
+  for (i = 0; i < nthreads; i++) pthread_create(&th[i], NULL, gemm_worker, &job);
+  for (i = 0; i < nthreads; i++) pthread_join(th[i], NULL);
+  return 0;
+}
+
+/* xorsum of n 32-bit words (AEGIS fingerprint, R6). */
+uint32_t orc_xorsum(const uint32_t *w, size_t n) {
+  uint32_t r = 0;
+  size_t i;
+  for (i = 0; i < n; i++) r ^= w[i];
+  return r;
+}
+
+/* Per-tile fingerprints of D [M][N]: fp[(i/16)*(N/16) + j/16] = xorsum of
+ * the 16x16 tile at (i, j). */
+void orc_tile_fingerprints(const uint32_t *D, int M, int N, uint32_t *fp) {
+  int i, j, r, c;
+  for (i = 0; i < M; i += 16)
+    for (j = 0; j < N; j += 16) {
+      uint32_t x = 0;
+      for (r = 0; r < 16; r++)
+        for (c = 0; c < 16; c++) x ^= D[(size_t)(i + r) * N + j + c];
+      fp[(size_t)(i / 16) * (N / 16) + j / 16] = x;
+    }
+}

@@ -1,0 +1,328 @@
+"""Benchmark: emulated MACs/s of the 4096^3 FP16-Ampere bit-exact GEMM.
+
+One step = one mmaemu_gemm call on the 4096x4096x4096 Ampere-FP16 workload
+(A, B fp16 ~ N(0,1), C = +0, per-16x16-tile xorsum fingerprints), i.e. the
+whole hot path: operand staging and decode, exact products, per-group max
+exponent, truncating alignment and signed sum, Ampere stage hand-over,
+toward-zero write-back, the 256-chunk K chain and the fused fingerprint
+epilogue.  Inputs are resident in HBM before timing starts; the 192 MiB
+working set (A 32 MiB, B 32 MiB, C 64 MiB, D 64 MiB) is larger than the
+126 MB L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With --gpus N > 1 launch it under torchrun: every rank runs its own
+4096^3 problem on its own GPU (weak scaling, the work partitions into
+independent problems, no data-path collective); the reported time is the max
+over ranks and ``value`` counts the MACs of all ranks.
+
+``--impl reference`` times the CPU oracle (the plain C restatement of the
+model) on the host cores on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+M = N = K = 4096
+MACS_PER_STEP = M * N * K
+OPS_PER_MAC = 7  # algorithmic integer ops per emulated MAC
+METRIC = "emulated MACs/s for 4096^3 FP16-Ampere GEMM; % of INT32-ALU roofline; bit-exact"
+UNIT = "MAC/s"
+# Pages' CPU simulator, same workload: 50.8 s per 4096x4096 FP16-Ampere MatMul
+# (K = 4096) on an Apple M4 Pro -> 68.72e9 / 50.8 MAC/s.  Context, not a target.
+PAGES_MACS_PER_S = MACS_PER_STEP / 50.8
+# ALU issue ceiling: 148 SMs x 4 SMSPs x 32 lanes at the 1965 MHz max SM clock.
+SMS, LANES_PER_SM, MAX_SM_MHZ = 148, 128, 1965.0
+ALU_PEAK_TOPS = SMS * LANES_PER_SM * MAX_SM_MHZ * 1e6 / 1e12
+H2D_BYTES = M * K * 2 + K * N * 2 + M * N * 4
+D2H_BYTES = M * N * 4 + (M // 16) * (N // 16) * 4
+WORKLOAD = "gemm M=N=K=4096, Ampere FP16 model, fp32 C=0 and D, fused per-16x16-tile xorsum"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ---------------------------------------------------------------------------
+# clocks sampling during the timed region
+# ---------------------------------------------------------------------------
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mmaemu_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4], parts[5:9]))
+            except ValueError:
+                continue
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[4]) if v.lower() == "active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+def clocks_bad(cl):
+    if any(r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown") for r in cl.get("reasons", [])):
+        return True
+    if cl.get("sm_mhz") and cl.get("sm_max_mhz") and not cl.get("reasons"):
+        return cl["sm_mhz"] < 0.6 * cl["sm_max_mhz"]
+    return False
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_rows(rows: int, nthreads: int, inputs=None):
+    from oracle import cref
+    from bit_exact_tensor_b200 import workloads as wl
+
+    A, B, C = inputs if inputs is not None else wl.config3()
+    t0 = time.perf_counter()
+    cref.gemm("ampere", "fp16", A, B, C, rows=(0, rows), nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(target_s: float = 12.0, inputs=None):
+    """Time the oracle as it stands on a bounded sample: the first R output
+    rows of the same GEMM (R x 4096 x 4096 MACs), R sized for ~target_s."""
+    from oracle import cref
+
+    nthreads = cref.default_threads()
+    rows = max(1, nthreads // 4)
+    dt = oracle_rows(rows, nthreads, inputs)
+    est = dt / rows
+    rows = int(max(1, min(M, target_s / max(est, 1e-6))))
+    dt = oracle_rows(rows, nthreads, inputs)
+    macs = rows * N * K
+    return {"value": macs / dt, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": f"output rows [0,{rows}) of the 4096^3 FP16-Ampere GEMM ({macs:.3e} MACs) "
+                      f"by the plain-C oracle, {nthreads} threads, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from oracle import cref
+    from bit_exact_tensor_b200 import workloads as wl
+
+    inputs = wl.config3()
+    nthreads = cref.default_threads()
+    steps, warmup = args.steps, args.warmup
+    budget = 150.0  # seconds for the whole run
+    probe = oracle_rows(max(1, nthreads // 4), nthreads, inputs) / max(1, nthreads // 4)
+    rows = int(max(1, min(M, budget / (steps + warmup) / max(probe, 1e-6))))
+    for _ in range(warmup):
+        oracle_rows(rows, nthreads, inputs)
+    times = [oracle_rows(rows, nthreads, inputs) for _ in range(steps)]
+    tot = sum(times)
+    macs = rows * N * K * steps
+    value = macs / tot
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": warmup, "ms_per_step": 1e3 * tot / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": value / PAGES_MACS_PER_S, "dtype": "int64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "sample_rows_per_step": rows},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                             "sample": f"output rows [0,{rows}) per step of the 4096^3 FP16-Ampere GEMM"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args):
+    import numpy as np
+    import torch
+
+    import bit_exact_tensor_b200 as mmaemu
+    from bit_exact_tensor_b200 import workloads as wl
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    A_np, B_np, C_np = wl.config3(seed=3 + 1000 * rank)
+    A = torch.from_numpy(A_np.view(np.int16)).to(dev)
+    B = torch.from_numpy(B_np.view(np.int16)).to(dev)
+    C = torch.from_numpy(C_np.view(np.int32)).to(dev)
+    D = torch.empty((M, N), dtype=torch.float32, device=dev)
+    fp = torch.empty(((M // 16) * (N // 16),), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mmaemu.gemm("ampere", "fp16", A, B, C, out=D, fp_out=fp)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    def timed():
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for s, e in ev:
+            s.record(stream)
+            step()
+            e.record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        per = [s.elapsed_time(e) for s, e in ev]
+        return t0.elapsed_time(t1), per
+
+    with ClockSampler(local) as cs:
+        total_ms, per_ms = timed()
+    clocks = cs.summary()
+    if clocks_bad(clocks):
+        with ClockSampler(local) as cs:
+            total_ms, per_ms = timed()
+        clocks = cs.summary()
+        clocks["remeasured"] = True
+    total_ms = max_over_ranks(total_ms)
+    kern_ms = max_over_ranks(sum(per_ms) / len(per_ms))
+
+    # end to end through the public API from pinned host buffers
+    A_h = torch.from_numpy(A_np.view(np.int16)).pin_memory()
+    B_h = torch.from_numpy(B_np.view(np.int16)).pin_memory()
+    C_h = torch.from_numpy(C_np.view(np.int32)).pin_memory()
+    mmaemu.gemm_host("ampere", "fp16", A_h, B_h, C_h, device=dev)  # warm-up
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        D_h, fp_h = mmaemu.gemm_host("ampere", "fp16", A_h, B_h, C_h, device=dev)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps)
+    barrier()
+
+    if rank == 0:
+        value = MACS_PER_STEP * world / (total_ms / 1e3 / args.steps)
+        achieved = OPS_PER_MAC * MACS_PER_STEP / (kern_ms / 1e3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": value / PAGES_MACS_PER_S, "dtype": "int32",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "emulated_arch": "ampere",
+                       "input_format": "fp16", "global_batch": world, "parallelism": f"independent x{world}",
+                       "l2": "inputs larger than L2 (192 MiB working set per GPU)"},
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": ALU_PEAK_TOPS, "unit": "Tops/s",
+                         "frac": achieved / ALU_PEAK_TOPS, "traffic": None,
+                         "kernel": "gemm_kernel<ampere,fp16>", "ops_per_mac": OPS_PER_MAC,
+                         "peak_basis": "148 SM x 128 lanes x 1965 MHz issue ceiling (derived)"},
+            "clocks": clocks,
+            "e2e": {"value": MACS_PER_STEP * world / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": H2D_BYTES, "d2h_bytes_per_step": D2H_BYTES},
+            "gpu_launches": args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(inputs=(A_np, B_np, C_np))
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

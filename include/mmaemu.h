@@ -1,0 +1,109 @@
+/*
+ * libmmaemu -- bit-exact emulation of other GPUs' Tensor Core MMA arithmetic
+ * on B200 (sm_100a) CUDA cores.  C ABI, no C++ or framework types.
+ *
+ * The arithmetic follows the characterise-then-simulate models recovered in
+ * "Hawkeye: Reproducing GPU-Level Non-Determinism (MLSys 2026)" (reading
+ * notes): Key observations Obs. 1-4, the target-test table, the recovered
+ * Ampere FP16 pipeline (Algorithms 12-14, Figure 1) with its Hopper and BF16
+ * paragraphs, and Algorithm 10 (BF16 extended range).  The per-tile
+ * fingerprint is the xorsum of "How AEGIS Turns Training Redundancy into
+ * Evidence" (AEGIS chapter 6, "Redundancy already exists in the training
+ * computation").
+ *
+ * Common rules for every call below:
+ *  - All data pointers are DEVICE pointers owned by the caller; the library
+ *    never frees, keeps or writes outside them.  Inputs are never modified.
+ *  - Matrices are dense and row-major.  fp16 and bf16 elements are 2 bytes,
+ *    e4m3 elements 1 byte (OCP FP8 E4M3: no infinities, S.1111.111 is NaN),
+ *    C and D are IEEE fp32.  Every pointer must be 16-byte aligned.
+ *  - Work is enqueued on the stream set with mmaemu_set_stream for the
+ *    calling host thread (default: the legacy default stream) and is
+ *    asynchronous unless stated otherwise.  Errors of the kernels themselves
+ *    surface at the caller's next synchronisation, or at mmaemu_xorsum.
+ *  - Results are fully deterministic: the same inputs give the same bits on
+ *    every run, whatever the stream or launch history.
+ *  - Return value: MMAEMU_OK (0) or a negative MMAEMU_E* code;
+ *    mmaemu_strerror gives a message.
+ */
+#ifndef MMAEMU_H
+#define MMAEMU_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Arithmetic models (Obs. 2 and Obs. 3).
+ *  MMAEMU_AMPERE: 24-bit internal significand; two accumulation stages,
+ *                 {C, P[1..8]} then {stage-1 result, P[9..16]}.  The pages
+ *                 also report Lovelace as identical to Ampere.
+ *  MMAEMU_HOPPER: 25-bit internal significand; one 17-term stage
+ *                 {C, P[1..16]}.                                           */
+enum { MMAEMU_AMPERE = 0, MMAEMU_HOPPER = 1 };
+
+/* Input formats.  E4M3 exists only with MMAEMU_HOPPER (FP8 is characterised
+ * on Hopper only; Ampere has no FP8 MMA).                                   */
+enum { MMAEMU_FP16 = 0, MMAEMU_BF16 = 1, MMAEMU_E4M3 = 2 };
+
+/* Return codes. */
+#define MMAEMU_OK 0
+#define MMAEMU_EINVAL (-1)       /* bad enum or pair, NULL or misaligned pointer, bad size */
+#define MMAEMU_ECUDA (-2)        /* a CUDA runtime call or launch failed                    */
+#define MMAEMU_ETIMEOUT (-3)     /* a bounded device wait gave up (reserved; no call waits) */
+#define MMAEMU_EUNSUPPORTED (-4) /* the current device is not an sm_100 GPU                 */
+
+/* Select the CUDA stream (a cudaStream_t passed as void*) that the calling
+ * host thread's later calls enqueue on; NULL selects the legacy default
+ * stream.  The setting is per host thread.  Never fails: returns MMAEMU_OK. */
+int mmaemu_set_stream(void *cuda_stream);
+
+/* Independent tile MMAs: for t < ntiles, D[t] = C[t] + A[t] . B[t] on
+ * 16x16x16 tiles, every element following the model's arithmetic (exact
+ * unnormalised products, truncating alignment to the group's largest
+ * exponent, the model's accumulation stages, toward-zero write-back with
+ * overflow to +-Inf) -- Obs. 1-3; recovered pipeline.
+ *   A: [ntiles][16][16] in fmt, element (m, k) of tile t at A[t*256 + m*16 + k]
+ *   B: [ntiles][16][16] in fmt, element (k, n) at B[t*256 + k*16 + n]
+ *   C: [ntiles][16][16] fp32 (m, n), or NULL for +0 everywhere
+ *   D: [ntiles][16][16] fp32 (m, n); D may equal C (in place); no other overlap
+ * ntiles == 0 is a no-op.  Errors: MMAEMU_EINVAL, MMAEMU_ECUDA,
+ * MMAEMU_EUNSUPPORTED; on error nothing is enqueued.                        */
+int mmaemu_tiles(int model, int fmt, const void *A, const void *B, const float *C, float *D,
+                 size_t ntiles);
+
+/* Large MatMul composed of 16x16x16 tiles (Obs. 4): D = C + A . B where K is
+ * walked in 16-wide chunks in ascending order and the fp32 result of each
+ * chunk is the C of the next, so every output element is
+ *   d_0 = C[m][n];  d_{j+1} = MMA16(A[m][16j..16j+15], B[16j..16j+15][n], d_j).
+ *   A: [M][K] in fmt; B: [K][N] in fmt; C, D: [M][N] fp32; C may be NULL (+0)
+ *   and may equal D (in place); no other overlap.
+ *   M, N, K: positive multiples of 16, M*K, K*N and M*N below 2^31.
+ *   fingerprint_out: NULL, or [(M/16)*(N/16)] uint32 written with the
+ *   xorsum (XOR of the 256 fp32 bit patterns) of each 16x16 tile of D, tiles
+ *   in row-major tile-grid order -- the AEGIS xorsum fingerprint, fused into
+ *   the epilogue.
+ * Errors: MMAEMU_EINVAL, MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED; on error nothing
+ * is enqueued.                                                              */
+int mmaemu_gemm(int model, int fmt, int M, int N, int K, const void *A, const void *B,
+                const float *C, float *D, uint32_t *fingerprint_out);
+
+/* xorsum of n 32-bit words at device pointer D (the AEGIS fingerprint of a
+ * whole tensor), written to *out_host.  SYNCHRONOUS: returns after the
+ * result is on the host (it waits for the selected stream).  n == 0 gives 0.
+ * Uses a few bytes of stream-ordered scratch that it releases before
+ * returning.  Errors: MMAEMU_EINVAL (NULL pointer, misaligned D),
+ * MMAEMU_ECUDA (also reports an earlier asynchronous kernel fault),
+ * MMAEMU_EUNSUPPORTED.                                                      */
+int mmaemu_xorsum(const void *D, size_t n, uint32_t *out_host);
+
+/* Static message for a return code. */
+const char *mmaemu_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MMAEMU_H */

@@ -1,0 +1,100 @@
+"""The C-ABI library loads, exports what include/mmaemu.h declares and rejects
+bad arguments before touching a device (CPU only; no compute calls)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mmaemu.h")
+
+
+def header_text():
+    return open(HEADER).read()
+
+
+def declared_functions():
+    src = re.sub(r"/\*.*?\*/", "", header_text(), flags=re.S)
+    return sorted(set(re.findall(r"\b(mmaemu_[a-z_0-9]+)\s*\(", src)))
+
+
+def declared_constants():
+    consts = {}
+    for name, val in re.findall(r"#define\s+(MMAEMU_[A-Z_0-9]+)\s+\(?(-?\d+)\)?", header_text()):
+        consts[name] = int(val)
+    for body in re.findall(r"enum\s*\{([^}]*)\}", re.sub(r"/\*.*?\*/", "", header_text(), flags=re.S)):
+        for name, val in re.findall(r"(MMAEMU_[A-Z_0-9]+)\s*=\s*(-?\d+)", body):
+            consts[name] = int(val)
+    return consts
+
+
+@pytest.fixture(scope="module")
+def L():
+    import bit_exact_tensor_b200 as m
+    from bit_exact_tensor_b200 import _build
+
+    _build.build_library()
+    return m.lib()
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == ["mmaemu_gemm", "mmaemu_set_stream", "mmaemu_strerror", "mmaemu_tiles",
+                                    "mmaemu_xorsum"]
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_constants_match_python_binding():
+    import bit_exact_tensor_b200 as m
+
+    c = declared_constants()
+    assert c["MMAEMU_AMPERE"] == m.MODELS["ampere"] and c["MMAEMU_HOPPER"] == m.MODELS["hopper"]
+    assert c["MMAEMU_FP16"] == m.FORMATS["fp16"] and c["MMAEMU_BF16"] == m.FORMATS["bf16"]
+    assert c["MMAEMU_E4M3"] == m.FORMATS["e4m3"]
+    assert (c["MMAEMU_OK"], c["MMAEMU_EINVAL"], c["MMAEMU_ECUDA"], c["MMAEMU_ETIMEOUT"],
+            c["MMAEMU_EUNSUPPORTED"]) == (0, -1, -2, -3, -4)
+
+
+def test_strerror_and_set_stream(L):
+    for code in (0, -1, -2, -3, -4, 7):
+        assert L.mmaemu_strerror(code)
+    assert L.mmaemu_set_stream(None) == 0
+
+
+def test_invalid_arguments_rejected_before_any_device_work(L):
+    EINVAL = -1
+    buf = ctypes.create_string_buffer(4096 + 16)
+    p = (ctypes.addressof(buf) + 15) & ~15
+    # bad enums, Ampere x E4M3, bad shapes, NULL and misaligned pointers
+    assert L.mmaemu_gemm(2, 0, 16, 16, 16, p, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(0, 3, 16, 16, 16, p, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(0, 2, 16, 16, 16, p, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(1, 0, 16, 24, 16, p, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(1, 0, 0, 16, 16, p, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(1, 0, 16, 16, -16, p, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(1, 0, 16, 16, 16, None, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(1, 0, 16, 16, 16, p + 2, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(1, 0, 1 << 16, 1 << 16, 16, p, p, None, p, None) == EINVAL
+    assert L.mmaemu_tiles(0, 2, p, p, None, p, 1) == EINVAL
+    assert L.mmaemu_tiles(0, 0, p, p, None, None, 1) == EINVAL
+    assert L.mmaemu_tiles(0, 0, p, p, p + 4, p, 1) == EINVAL
+    assert L.mmaemu_tiles(0, 0, p, p, None, p, 0) == 0  # empty batch is a no-op
+    assert L.mmaemu_xorsum(p, 4, None) == EINVAL
+    assert L.mmaemu_xorsum(p + 4, 4, ctypes.byref(ctypes.c_uint32())) == EINVAL
+
+
+def test_product_path_never_imports_the_oracle():
+    """The library package must not route through the CPU oracle."""
+    pkg = os.path.join(ROOT, "bit_exact_tensor_b200")
+    pat = re.compile(r"\b(import|from)\s+oracle\b|liborc|mmaemu_ref|\bcref\b|\borc_[a-z]")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not pat.search(text), f

@@ -1,0 +1,158 @@
+"""mmaemu_gemm on the GPU against the C oracle, bit for bit.
+
+Small and ragged shapes are compared element by element in full; the
+full-size workloads (4096^3 FP16-Ampere, 4096^3 BF16-Hopper with and without
+out-of-range sums, 8192x4096x14336 E4M3-Hopper) run in the same launch
+configuration the benchmark times and are checked on whole sampled rows,
+columns and random elements, plus fingerprints against the xorsum of D.
+"""
+
+import zlib
+
+import numpy as np
+import pytest
+
+from bit_exact_tensor_b200 import workloads as wl
+from gpu_util import dev_f32, dev_in, first_mismatch, host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gemm(model, fmt, A, B, C, fingerprint=True):
+    import bit_exact_tensor_b200 as mmaemu
+
+    D, fp = mmaemu.gemm(model, fmt, dev_in(A), dev_in(B), dev_f32(C) if C is not None else None,
+                        fingerprint=fingerprint)
+    return host_bits(D), (host_bits(fp) if fp is not None else None)
+
+
+def normal_inputs(M, N, K, fmt, seed):
+    rng = np.random.default_rng(seed)
+    A = wl.to_bits(rng.standard_normal((M, K)), fmt)
+    B = wl.to_bits(rng.standard_normal((K, N)), fmt)
+    C = wl.f32_bits(rng.standard_normal((M, N)))
+    for X in (A, B):
+        pick = rng.random(X.shape) < 0.05
+        X[pick] = wl.random_subnormals(rng, X.shape, fmt)[pick]
+    return A, B, C
+
+
+SHAPES = [(16, 16, 16), (64, 128, 32), (80, 144, 48), (208, 272, 160), (128, 16, 512), (16, 400, 96)]
+
+
+@pytest.mark.parametrize("model,fmt", wl.PAIRS)
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_small_and_ragged_full_compare(cref, model, fmt, shape):
+    M, N, K = shape
+    A, B, C = normal_inputs(M, N, K, fmt, seed=M * 7 + N * 3 + K)
+    D, fp = run_gemm(model, fmt, A, B, C)
+    want = cref.gemm(model, fmt, A, B, C)
+    assert np.array_equal(D, want), first_mismatch(D, want)
+    assert np.array_equal(fp, cref.tile_fingerprints(want))
+
+
+@pytest.mark.parametrize("model,fmt", wl.PAIRS)
+def test_specials_in_the_k_chain(cref, model, fmt):
+    """NaN / Inf / signed zeros in A, B and C, and C = +-Inf or NaN carried
+    through later chunks."""
+    M, N, K = 48, 160, 80
+    A, B, C = normal_inputs(M, N, K, fmt, seed=17)
+    rng = np.random.default_rng(18)
+    sp = wl.special_patterns(fmt)
+    for X in (A, B):
+        pick = rng.random(X.shape) < 0.01
+        X[pick] = sp[rng.integers(0, sp.size, size=int(pick.sum()))]
+    pick = rng.random(C.shape) < 0.05
+    C[pick] = np.array([0x7F800000, 0xFF800000, 0x7FC00001, 0x80000000, 0x00000001],
+                       dtype=np.uint32)[rng.integers(0, 5, size=int(pick.sum()))]
+    D, fp = run_gemm(model, fmt, A, B, C)
+    want = cref.gemm(model, fmt, A, B, C)
+    assert np.array_equal(D, want), first_mismatch(D, want)
+
+
+def test_null_c_in_place_and_no_fingerprint(cref):
+    import bit_exact_tensor_b200 as mmaemu
+
+    A, B, C = normal_inputs(96, 96, 64, "fp16", seed=3)
+    D, fp = run_gemm("ampere", "fp16", A, B, None, fingerprint=False)
+    assert fp is None
+    assert np.array_equal(D, cref.gemm("ampere", "fp16", A, B, None))
+    Ct = dev_f32(C)
+    mmaemu.gemm("ampere", "fp16", dev_in(A), dev_in(B), Ct, out=Ct, fingerprint=False)
+    assert np.array_equal(host_bits(Ct), cref.gemm("ampere", "fp16", A, B, C))
+
+
+def test_gemm_k16_equals_tiles_and_k_split(cref):
+    import bit_exact_tensor_b200 as mmaemu
+
+    A, B, C = normal_inputs(16, 16, 16, "bf16", seed=4)
+    D, _ = run_gemm("hopper", "bf16", A, B, C)
+    Dt = mmaemu.tiles("hopper", "bf16", dev_in(A.reshape(1, 16, 16)), dev_in(B.reshape(1, 16, 16)),
+                      dev_f32(C.reshape(1, 16, 16)))
+    assert np.array_equal(D, host_bits(Dt).reshape(16, 16))
+    A, B, C = normal_inputs(64, 128, 96, "fp16", seed=5)
+    D, _ = run_gemm("ampere", "fp16", A, B, C)
+    D1, _ = run_gemm("ampere", "fp16", A[:, :48].copy(), B[:48].copy(), C)
+    D2, _ = run_gemm("ampere", "fp16", A[:, 48:].copy(), B[48:].copy(), D1)
+    assert np.array_equal(D, D2)
+
+
+def test_bad_arguments_raise():
+    import torch
+
+    import bit_exact_tensor_b200 as mmaemu
+
+    A = torch.zeros((32, 32), dtype=torch.float16, device="cuda")
+    with pytest.raises(mmaemu.MmaEmuError):
+        mmaemu.gemm("ampere", "fp16", A[:, :24].contiguous(), torch.zeros((24, 32), dtype=torch.float16,
+                                                                        device="cuda"))
+    A8 = torch.zeros((32, 32), dtype=torch.uint8, device="cuda")
+    with pytest.raises(mmaemu.MmaEmuError):
+        mmaemu.gemm("ampere", "e4m3", A8, A8)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled
+# ---------------------------------------------------------------------------
+
+FULL = {
+    "cfg3-ampere-fp16-4096": ("ampere", "fp16", lambda: wl.config3()),
+    "cfg4-hopper-bf16-4096": ("hopper", "bf16", lambda: wl.config4()),
+    "cfg4b-hopper-bf16-4096-wide": ("hopper", "bf16", lambda: wl.config4(wide=True)),
+    "cfg5-hopper-e4m3-8192x4096x14336": ("hopper", "e4m3", lambda: wl.config5()),
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_size_sampled(cref, name):
+    model, fmt, make = FULL[name]
+    A, B, C = make()
+    M, K = A.shape
+    N = B.shape[1]
+    D, fp = run_gemm(model, fmt, A, B, C)
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    # whole rows and columns at the edges and inside, and random elements
+    rows = [0, M - 1, int(rng.integers(1, M - 1))]
+    cols = [0, N - 1, int(rng.integers(1, N - 1))]
+    for r in rows:
+        want = cref.gemm(model, fmt, A, B, C, rows=(r, r + 1))[r]
+        assert np.array_equal(D[r], want), (name, "row", r, first_mismatch(D[r], want))
+    for c in cols:
+        want = cref.gemm(model, fmt, A, B, C, cols=(c, c + 1))[:, c]
+        assert np.array_equal(D[:, c], want), (name, "col", c, first_mismatch(D[:, c], want))
+    for _ in range(64):
+        m, n = int(rng.integers(0, M)), int(rng.integers(0, N))
+        assert D[m, n] == cref.gemm_element(model, fmt, A, B, C, m, n), (name, m, n)
+    # fingerprints: xorsum of every 16x16 tile of the GPU's D, all tiles
+    t = D.reshape(M // 16, 16, N // 16, 16)
+    fp_host = np.bitwise_xor.reduce(np.bitwise_xor.reduce(t, axis=3), axis=1).reshape(-1)
+    assert np.array_equal(fp, fp_host)
+    if name.startswith("cfg4b"):
+        assert (D == 0x7F800000).any() and (D == 0xFF800000).any()  # the sums left fp32 range
+
+
+def test_full_size_deterministic():
+    A, B, C = wl.config3()
+    _, fp1 = run_gemm("ampere", "fp16", A, B, C)
+    _, fp2 = run_gemm("ampere", "fp16", A, B, C)
+    assert np.array_equal(fp1, fp2)

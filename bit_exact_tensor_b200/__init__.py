@@ -15,7 +15,7 @@ import ctypes
 import os
 import threading
 
-__all__ = ["MODELS", "FORMATS", "MmaEmuError", "lib", "tiles", "gemm", "xorsum", "gemm_host",
+__all__ = ["MODELS", "FORMATS", "MmaEmuError", "lib", "tiles", "gemm", "xorsum", "xorsum_noalloc", "gemm_host",
            "set_stream"]
 
 MODELS = {"ampere": 0, "hopper": 1}
@@ -202,3 +202,32 @@ def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bo
         fp_host.copy_(fp, non_blocking=True)
     torch.cuda.current_stream().synchronize()
     return D_host, fp_host
+
+
+def xorsum_noalloc(t) -> int:
+    """Same value as :func:`xorsum`, computed without allocating any device
+    memory: the library keeps a fixed scratch array for it.  Meant for code
+    that cannot allocate when it needs the fingerprint (for instance a check
+    that runs after the device ran out of memory, or a process whose device
+    memory is fully reserved by another allocator).  At most 2^27 words;
+    concurrent calls on different streams must not overlap (they share the
+    scratch).  Synchronous."""
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+        raise TypeError("xorsum_noalloc needs a contiguous CUDA tensor")
+    nbytes = t.numel() * t.element_size()
+    if nbytes % 4:
+        raise ValueError("tensor size must be a whole number of 32-bit words")
+    if nbytes // 4 > NOALLOC_MAX_WORDS:
+        raise ValueError(f"xorsum_noalloc handles at most {NOALLOC_MAX_WORDS} words (its fixed scratch "
+                         f"limit); got {nbytes // 4}")
+    fn = lib().mmaemu_xorsum_noalloc
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32)]
+    fn.restype = ctypes.c_int
+    res = ctypes.c_uint32(0)
+    set_stream()
+    _check(fn(t.data_ptr(), nbytes // 4, ctypes.byref(res)), "mmaemu_xorsum_noalloc")
+    return int(res.value)
+
+
+NOALLOC_MAX_WORDS = 1 << 27  # MMAEMU_XORSUM_NOALLOC_MAX_WORDS

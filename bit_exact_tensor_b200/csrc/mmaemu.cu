@@ -619,3 +619,122 @@ const char *mmaemu_strerror(int code) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// xorsum that allocates nothing
+//
+// For callers that cannot allocate device memory at the moment they need a
+// fingerprint -- for instance a checker that runs after the device has run out
+// of memory, or inside a process whose device memory is entirely reserved by
+// another allocator -- mmaemu_xorsum_noalloc does the same reduction with a
+// fixed scratch array that lives in the library image instead of a per-call
+// allocation.  Each block of xorsum_partials_kernel folds a fixed span of the
+// input into one word of the array; xorsum_finish_kernel folds those words
+// into the result slot, which is then copied to the host.
+// ===========================================================================
+namespace mmaemu {
+
+constexpr unsigned kNoAllocThreads = 256;
+constexpr size_t kNoAllocVecPerThread = 8;  // uint4 loads per thread
+constexpr size_t kNoAllocVecPerBlock = kNoAllocThreads * kNoAllocVecPerThread;
+constexpr size_t kNoAllocWordsPerBlock = 4 * kNoAllocVecPerBlock;  // 8192 words
+constexpr size_t kNoAllocPartials = MMAEMU_XORSUM_NOALLOC_MAX_WORDS / kNoAllocWordsPerBlock;  // 16384
+static_assert(kNoAllocPartials * kNoAllocWordsPerBlock == MMAEMU_XORSUM_NOALLOC_MAX_WORDS, "exact fit");
+
+// One word per block, then the result slot.  Every word a call reads has been
+// written earlier in the same call, so nothing needs clearing between calls.
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocPartials + 1];
+
+__global__ void __launch_bounds__(kNoAllocThreads) xorsum_partials_kernel(const uint4 *__restrict__ v, size_t nvec,
+                                                                          const uint32_t *__restrict__ tail,
+                                                                          int ntail, uint32_t *__restrict__ partials) {
+  __shared__ uint32_t part[kNoAllocThreads / 32];
+  uint32_t x = 0;
+  const size_t base = (size_t)blockIdx.x * kNoAllocVecPerBlock;
+#pragma unroll
+  for (size_t i = 0; i < kNoAllocVecPerThread; i++) {
+    const size_t idx = base + i * kNoAllocThreads + threadIdx.x;
+    if (idx < nvec) {
+      const uint4 q = v[idx];
+      x ^= q.x ^ q.y ^ q.z ^ q.w;
+    }
+  }
+  if (blockIdx.x == 0 && (int)threadIdx.x < ntail) x ^= tail[threadIdx.x];
+  x = __reduce_xor_sync(0xFFFFFFFFu, x);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = x;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t y = 0;
+    for (unsigned w = 0; w < kNoAllocThreads / 32; w++) y ^= part[w];
+    partials[blockIdx.x] = y;
+  }
+}
+
+__global__ void __launch_bounds__(kNoAllocThreads) xorsum_finish_kernel(const uint32_t *__restrict__ partials,
+                                                                        unsigned nparts, uint32_t *__restrict__ result) {
+  __shared__ uint32_t part[kNoAllocThreads / 32];
+  uint32_t x = 0;
+  for (unsigned i = threadIdx.x; i < nparts; i += kNoAllocThreads) x ^= partials[i];
+  x = __reduce_xor_sync(0xFFFFFFFFu, x);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = x;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t y = 0;
+    for (unsigned w = 0; w < kNoAllocThreads / 32; w++) y ^= part[w];
+    *result = y;
+  }
+}
+
+}  // namespace mmaemu
+
+namespace {
+
+// Device address of the scratch array, looked up once per device (with that
+// device current).  In host code the array's name only stands for the device
+// symbol; it is not an address a kernel may be given.
+std::atomic<uint32_t *> g_noalloc_scratch_ptr[kMaxDevices];
+
+int noalloc_scratch(uint32_t **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MMAEMU_ECUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MMAEMU_EUNSUPPORTED;
+  uint32_t *p = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), mmaemu::g_noalloc_scratch) != cudaSuccess ||
+        p == nullptr)
+      return MMAEMU_ECUDA;
+    g_noalloc_scratch_ptr[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return MMAEMU_OK;
+}
+
+}  // namespace
+
+extern "C" int mmaemu_xorsum_noalloc(const void *D, size_t n, uint32_t *out_host) {
+  if (!out_host || (n && !D) || (n && !aligned16(D))) return MMAEMU_EINVAL;
+  if (n > MMAEMU_XORSUM_NOALLOC_MAX_WORDS) return MMAEMU_EINVAL;
+  int rc = check_device();
+  if (rc != MMAEMU_OK) return rc;
+  uint32_t *scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc != MMAEMU_OK) return rc;
+  *out_host = 0;
+  if (n == 0) return MMAEMU_OK;
+  const size_t nvec = n / 4;
+  const int ntail = (int)(n % 4);
+  size_t nblocks = (nvec + mmaemu::kNoAllocVecPerBlock - 1) / mmaemu::kNoAllocVecPerBlock;
+  if (nblocks == 0) nblocks = 1;  // only the tail words
+  uint32_t *result_slot = scratch + mmaemu::kNoAllocPartials;
+  mmaemu::xorsum_partials_kernel<<<(unsigned)nblocks, mmaemu::kNoAllocThreads, 0, t_stream>>>(
+      static_cast<const uint4 *>(D), nvec, static_cast<const uint32_t *>(D) + 4 * nvec, ntail, scratch);
+  if (cudaGetLastError() != cudaSuccess) return MMAEMU_ECUDA;
+  mmaemu::xorsum_finish_kernel<<<1, mmaemu::kNoAllocThreads, 0, t_stream>>>(scratch, (unsigned)nblocks, result_slot);
+  if (cudaGetLastError() != cudaSuccess) return MMAEMU_ECUDA;
+  uint32_t result = 0;
+  if (cudaMemcpyAsync(&result, result_slot, sizeof(uint32_t), cudaMemcpyDeviceToHost, t_stream) != cudaSuccess)
+    return MMAEMU_ECUDA;
+  if (cudaStreamSynchronize(t_stream) != cudaSuccess) return MMAEMU_ECUDA;
+  *out_host = result;
+  return MMAEMU_OK;
+}

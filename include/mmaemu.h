@@ -99,6 +99,26 @@ int mmaemu_gemm(int model, int fmt, int M, int N, int K, const void *A, const vo
  * MMAEMU_EUNSUPPORTED.                                                      */
 int mmaemu_xorsum(const void *D, size_t n, uint32_t *out_host);
 
+/* mmaemu_xorsum for callers that cannot allocate device memory when they
+ * need the fingerprint -- e.g. a checker that must still run after the device
+ * has run out of memory, or a process whose device memory is wholly reserved
+ * by another allocator.  It has no counterpart on the pages; it computes the
+ * same value as mmaemu_xorsum.
+ *   Scratch: a fixed array inside the library (64 KiB + 4 bytes per GPU,
+ *   held by every GPU that loads the library until the process exits); no
+ *   cudaMalloc, cudaFree or other allocating call is made.
+ *   Limit: n <= MMAEMU_XORSUM_NOALLOC_MAX_WORDS (2^27 words = 512 MiB);
+ *   larger n returns MMAEMU_EINVAL before any device work.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the one array: calls whose work overlaps on the GPU (from
+ *   different streams or host threads) race and may return wrong values, so
+ *   serialise them.  Nothing in the array needs clearing between calls.
+ *   SYNCHRONOUS like mmaemu_xorsum.  Errors: MMAEMU_EINVAL, MMAEMU_ECUDA,
+ *   MMAEMU_EUNSUPPORTED.                                                    */
+#define MMAEMU_XORSUM_NOALLOC_MAX_WORDS ((size_t)1 << 27)
+int mmaemu_xorsum_noalloc(const void *D, size_t n, uint32_t *out_host);
+
 /* Static message for a return code. */
 const char *mmaemu_strerror(int code);
 

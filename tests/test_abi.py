@@ -41,7 +41,7 @@ def L():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == ["mmaemu_gemm", "mmaemu_set_stream", "mmaemu_strerror", "mmaemu_tiles",
-                                    "mmaemu_xorsum"]
+                                    "mmaemu_xorsum", "mmaemu_xorsum_noalloc"]
 
 
 def test_library_exports_every_declared_symbol(L):

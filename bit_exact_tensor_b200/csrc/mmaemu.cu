@@ -8,7 +8,9 @@
 //   xorsum_kernel -- XOR of a buffer of 32-bit words.
 // The arithmetic itself is in mmaemu_core.cuh; see the model citations there.
 // Tensor cores are deliberately not used: B200's own MMA arithmetic is not the
-// arithmetic being emulated, so everything is exact integer work.
+// arithmetic being emulated, so everything is exact integer work, balanced
+// between the ALU pipe (shifts, logic, min, add) and the IMAD pipe (products
+// and sign-carrying accumulation).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -22,16 +24,23 @@ namespace mmaemu {
 // ---------------------------------------------------------------------------
 // decoded operand panels in shared memory, [k][row] for A and [k][col] for B
 // ---------------------------------------------------------------------------
+// Each thread owns an R x CC block of outputs.  Its first NV3 columns apply
+// product signs with an IMAD by sigma_a * sigma_b (+-1); the others in ones'
+// complement with a per-group popcount correction.  bS therefore holds +-1
+// for columns n with n % CC < NV3 and a sign mask for the rest.
 template <int BM, int BN>
 struct __align__(16) Panel {
-  uint32_t aM[16][BM];  // ma << (F - 2p): one IMAD with mb gives the term magnitude
-  int32_t aN[16][BM];   // -ea (ZSENT / NINF / NNAN markers)
-  uint32_t aS[16][BM];  // sign masks
+  uint32_t aM[16][BM];   // ma << (F - 2p): one IMAD with mb gives the term magnitude
+  int32_t aN[16][BM];    // -ea (ZSENT / NINF / NNAN markers)
+  uint32_t aS[16][BM];   // sign mask (0 / all ones)
+  int32_t aP[16][BM];    // sign as +-1
+  uint32_t aN2[16][BM];  // (-ea, -ea) packed pair, for the packed max pass
   uint32_t bM[16][BN];
   int32_t bN[16][BN];
-  uint32_t bS[16][BN];
-  uint16_t sa16[BM];  // bit k = sign of a[m][k]
-  uint16_t sb16[BN];  // bit k = sign of b[k][n]
+  uint32_t bS[16][BN];   // +-1 or sign mask, by column class
+  int16_t bN2[16][BN];   // -eb as 16-bit: adjacent columns read as one pair
+  uint16_t sa16[BM];     // bit k = sign of a[m][k]
+  uint16_t sb16[BN];     // bit k = sign of b[k][n]
 };
 
 template <int R, typename T>
@@ -54,47 +63,54 @@ __device__ __forceinline__ void lds_vec(const T *p, T (&v)[R]) {
   }
 }
 
-// One accumulation group over k in [K0, K0 + KN): returns S (signed sum of
-// the aligned terms, carry term included) and nmin (= -e_max) per output.
-// The carry term is (nc, Xc) with Xc in ones' complement form.
-template <int FMT, int F, int K0, int KN, int R, int CC, int BM, int BN>
-__device__ __forceinline__ void group_sum(const Panel<BM, BN> &P, int rl, int cl,
-                                          const int32_t (&nc)[R][CC], const int32_t (&Xc)[R][CC],
-                                          int32_t (&nmin)[R][CC], int32_t (&S)[R][CC]) {
-  // pass 1: the group's max exponent (min of the negated exponents)
+// One accumulation group over k in [K0, K0 + KN) with a carried term given by
+// the state (Np, X): returns S (exact signed sum of the aligned terms) and
+// nmin (= -e_max) for every output.
+template <int FMT, int F, int K0, int KN, int R, int CC, int NV3, int BM, int BN>
+__device__ __forceinline__ void group_sum(const Panel<BM, BN> &P, int rl, int cl, const uint32_t (&Np)[R][CC / 2],
+                                          const int32_t (&X)[R][CC], int32_t (&nmin)[R][CC], int32_t (&S)[R][CC]) {
+  // pass 1: the group's max exponent, two outputs per packed instruction
+  uint32_t nm2[R][CC / 2];
 #pragma unroll
   for (int r = 0; r < R; r++)
 #pragma unroll
-    for (int c = 0; c < CC; c++) nmin[r][c] = nc[r][c];
+    for (int p = 0; p < CC / 2; p++) nm2[r][p] = Np[r][p];
 #pragma unroll 1
   for (int k = K0; k < K0 + KN; k++) {
-    int32_t an[R], bn[CC];
-    lds_vec<R>(&P.aN[k][rl], an);
-    lds_vec<CC>(&P.bN[k][cl], bn);
+    uint32_t an2[R], bn2[CC / 2];
+    lds_vec<R>(&P.aN2[k][rl], an2);
+    lds_vec<CC / 2>(reinterpret_cast<const uint32_t *>(&P.bN2[k][cl]), bn2);
 #pragma unroll
     for (int r = 0; r < R; r++)
 #pragma unroll
-      for (int c = 0; c < CC; c++) nmin[r][c] = min(nmin[r][c], an[r] + bn[c]);
+      for (int p = 0; p < CC / 2; p++) nm2[r][p] = vmin2(nm2[r][p], vadd2(an2[r], bn2[p]));
   }
-  if constexpr (kNeedsFloor<FMT>) {
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int c = 0; c < CC; c++) nmin[r][c] = min(nmin[r][c], NFLOOR);
-  }
-  // pass 2: align (truncate) and add; the carry first
 #pragma unroll
   for (int r = 0; r < R; r++)
 #pragma unroll
-    for (int c = 0; c < CC; c++)
-      S[r][c] = shr_s32(Xc[r][c], (uint32_t)(nc[r][c] - nmin[r][c])) + (int32_t)((uint32_t)Xc[r][c] >> 31);
+    for (int p = 0; p < CC / 2; p++) {
+      uint32_t v = nm2[r][p];
+      if constexpr (kNeedsFloor<FMT>) v = vmin2(v, (uint32_t)NFLOOR | ((uint32_t)NFLOOR << 16));
+      nmin[r][2 * p] = lo16(v);
+      nmin[r][2 * p + 1] = hi16(v);
+    }
+  // pass 2: the carried term, then each product aligned (truncated) and added
+  constexpr int CSH = 30 - F;  // the state's significand sits at bits 30..7
+#pragma unroll
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int c = 0; c < CC; c++) {
+      const int32_t nc = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
+      S[r][c] = shr_s32(X[r][c], (uint32_t)(nc - nmin[r][c] + CSH)) - (X[r][c] >> 31);
+    }
 #pragma unroll 1
   for (int k = K0; k < K0 + KN; k++) {
     uint32_t am[R], as[R], bm[CC], bs[CC];
-    int32_t an[R], bn[CC];
+    int32_t an[R], ap[R], bn[CC];
     lds_vec<R>(&P.aM[k][rl], am);
     lds_vec<R>(&P.aN[k][rl], an);
     lds_vec<R>(&P.aS[k][rl], as);
+    lds_vec<R>(&P.aP[k][rl], ap);
     lds_vec<CC>(&P.bM[k][cl], bm);
     lds_vec<CC>(&P.bN[k][cl], bn);
     lds_vec<CC>(&P.bS[k][cl], bs);
@@ -103,121 +119,244 @@ __device__ __forceinline__ void group_sum(const Panel<BM, BN> &P, int rl, int cl
 #pragma unroll
       for (int c = 0; c < CC; c++) {
         const uint32_t T = shr_u32(am[r] * bm[c], (uint32_t)(an[r] + bn[c] - nmin[r][c]));
-        S[r][c] += (int32_t)(T ^ as[r] ^ bs[c]);
+        if (c < NV3) {
+          S[r][c] += (int32_t)T * (ap[r] * (int32_t)bs[c]);
+        } else {
+          S[r][c] += (int32_t)(T ^ as[r] ^ bs[c]);
+        }
       }
   }
-  // ones' complement correction: + number of negative products in the group
+  // ones' complement columns: add back the number of negative products
+  if constexpr (NV3 < CC) {
 #pragma unroll
-  for (int r = 0; r < R; r++)
+    for (int r = 0; r < R; r++) {
+      const uint32_t sa = P.sa16[rl + r];
 #pragma unroll
-    for (int c = 0; c < CC; c++) {
-      const uint32_t neg = ((uint32_t)P.sa16[rl + r] ^ (uint32_t)P.sb16[cl + c]) >> K0;
-      S[r][c] += __popc(neg & ((1u << KN) - 1u));
+      for (int c = NV3; c < CC; c++) {
+        const uint32_t neg = ((sa ^ (uint32_t)P.sb16[cl + c]) >> K0) & ((1u << KN) - 1u);
+        S[r][c] += __popc(neg);
+      }
     }
+  }
 }
 
-// One 16-deep K chunk for an R x CC block of outputs at panel row rl, col cl.
-// D holds the fp32 accumulator input on entry and the result on exit.
-template <int MODEL, int FMT, int R, int CC, int BM, int BN>
-__device__ __forceinline__ void mma_chunk(const Panel<BM, BN> &P, int rl, int cl, uint32_t (&D)[R][CC],
-                                          bool panel_special) {
-  constexpr int F = ModelT<MODEL>::F;
-  static_assert(R * CC <= 32, "per-output bit masks hold 32 outputs");
-  uint32_t c_negzero = 0, c_nan = 0, c_infp = 0, c_infn = 0;
-  int32_t nc[R][CC], Xc[R][CC], nmin[R][CC], S[R][CC];
-#pragma unroll
-  for (int r = 0; r < R; r++)
-#pragma unroll
-    for (int c = 0; c < CC; c++) {
-      const uint32_t x = D[r][c], bit = 1u << (r * CC + c);
-      c_negzero |= (x == 0x80000000u) ? bit : 0u;
-      const bool sp = ((x >> 23) & 0xFFu) == 0xFFu;
-      c_nan |= (sp && (x & 0x7FFFFFu)) ? bit : 0u;
-      c_infp |= (x == 0x7F800000u) ? bit : 0u;
-      c_infn |= (x == 0xFF800000u) ? bit : 0u;
-      c_term<F>(x, nc[r][c], Xc[r][c]);
-    }
+// normalise a nonzero sum to the state form: X with its leading bit at bit 30,
+// and n = -(exponent of the leading bit)
+template <int F>
+__device__ __forceinline__ void to_state(int32_t s, int32_t nmin, int32_t &n, int32_t &X, uint32_t mask) {
+  const uint32_t mag = (uint32_t)(s < 0 ? -s : s);
+  const uint32_t z = __clz(mag);
+  const uint32_t M = shl_u32(mag, z);
+  n = nmin + (int32_t)z - (31 - F);
+  X = (int32_t)(((M >> 1) & mask) ^ (uint32_t)(s >> 31));
+}
 
-  if constexpr (MODEL == MODEL_AMPERE) {
-    // stage 1: {C, P[1..8]}
-    group_sum<FMT, F, 0, 8, R, CC>(P, rl, cl, nc, Xc, nmin, S);
-    // hand-over: the stage-1 sum normalised to 24 bits (truncated), exponent
-    // unbounded (BF16 extended range); a zero sum contributes no term
+// Special-value outcome of each output of an R x CC block whose chunk holds
+// Inf or NaN somewhere in its A or B panel: 2 bits per output (0 none, 1 NaN,
+// 2 +Inf, 3 -Inf).  c_nan / c_infp / c_infn flag outputs whose incoming value
+// is NaN / +Inf / -Inf.  Kept out of line: it is rare and would otherwise
+// crowd the registers of the main path.
+template <int R, int CC, int BM, int BN>
+__device__ __noinline__ uint64_t special_codes(const Panel<BM, BN> *P, int rl, int cl, uint32_t c_nan, uint32_t c_infp,
+                                               uint32_t c_infn) {
+  uint64_t codes = 0;
+#pragma unroll 1
+  for (int o = 0; o < R * CC; o++) {
+    const int r = o / CC, c = o % CC;
+    bool nan = (c_nan >> o) & 1u, ip = (c_infp >> o) & 1u, in = (c_infn >> o) & 1u;
+#pragma unroll 1
+    for (int k = 0; k < 16; k++) {
+      const int32_t an = P->aN[k][rl + r], bn = P->bN[k][cl + c];
+      if (an == NNAN || bn == NNAN) {
+        nan = true;
+      } else if (an == NINF || bn == NINF) {
+        if (an == ZSENT || bn == ZSENT) nan = true;
+        else if ((P->aS[k][rl + r] ^ P->bS[k][cl + c]) & 0x80000000u) in = true;
+        else ip = true;
+      }
+    }
+    const uint64_t code = (nan || (ip && in)) ? 1u : ip ? 2u : in ? 3u : 0u;
+    codes |= code << (2 * o);
+  }
+  return codes;
+}
+
+// One 16-deep K chunk for an R x CC block of outputs at panel row rl, col cl,
+// updating the accumulator state (Np, X, dneg0) in place.
+//   Np    -- n of adjacent output pairs, packed
+//   X     -- significands (see mmaemu_core.cuh)
+//   dneg0 -- bit r*CC+c set when that output's state is -0
+template <int MODEL, int FMT, int R, int CC, int NV3, int BM, int BN>
+__device__ __forceinline__ void mma_chunk(const Panel<BM, BN> &P, int rl, int cl, uint32_t (&Np)[R][CC / 2],
+                                          int32_t (&X)[R][CC], uint32_t &dneg0, bool panel_special) {
+  constexpr int F = ModelT<MODEL>::F;
+  static_assert(R * CC <= 32 && CC % 2 == 0, "per-output masks hold 32 outputs");
+  // the Hopper grid has 24 fraction bits: keep the state's bit 6 clear
+  constexpr uint32_t XMASK = F == 24 ? 0x7FFFFF80u : 0x7FFFFFFFu;
+
+  // kinds of the incoming values, needed only when A/B hold Inf or NaN
+  uint32_t c_nan = 0, c_infp = 0, c_infn = 0;
+  if (panel_special) {
 #pragma unroll
     for (int r = 0; r < R; r++)
 #pragma unroll
       for (int c = 0; c < CC; c++) {
-        const int32_t s = S[r][c];
-        const uint32_t mag = (uint32_t)(s < 0 ? -s : s);
-        const uint32_t z = __clz(mag);
-        const uint32_t M = shl_u32(mag, z) >> 8;
-        nc[r][c] = s ? nmin[r][c] - 8 + (int32_t)z : ZSENT;
-        Xc[r][c] = (int32_t)(M ^ (uint32_t)(s >> 31));
+        const int32_t n = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
+        const uint32_t bit = 1u << (r * CC + c);
+        if (n == STATE_NAN) c_nan |= bit;
+        if (n == STATE_INF) {
+          if (X[r][c] < 0) c_infn |= bit;
+          else c_infp |= bit;
+        }
       }
-    // stage 2: {S1, P[9..16]}
-    group_sum<FMT, F, 8, 8, R, CC>(P, rl, cl, nc, Xc, nmin, S);
-  } else {
-    // one stage: {C, P[1..16]}
-    group_sum<FMT, F, 0, 16, R, CC>(P, rl, cl, nc, Xc, nmin, S);
   }
 
-  // toward-zero write-back
+  int32_t S[R][CC], nmin[R][CC];
+  if constexpr (MODEL == MODEL_AMPERE) {
+    // stage 1: {C, P[1..8]}
+    group_sum<FMT, F, 0, 8, R, CC, NV3>(P, rl, cl, Np, X, nmin, S);
+    // hand-over: the stage-1 sum as a 24-bit term (the state form keeps extra
+    // low bits, but stage 2 shifts it right by at least 7, which truncates
+    // them exactly like the normalisation would); a zero sum adds no term
+#pragma unroll
+    for (int r = 0; r < R; r++)
+#pragma unroll
+      for (int p = 0; p < CC / 2; p++) {
+        int32_t n0, n1;
+        to_state<F>(S[r][2 * p], nmin[r][2 * p], n0, X[r][2 * p], 0x7FFFFFFFu);
+        to_state<F>(S[r][2 * p + 1], nmin[r][2 * p + 1], n1, X[r][2 * p + 1], 0x7FFFFFFFu);
+        Np[r][p] = pack16(S[r][2 * p] ? n0 : ZSENT, S[r][2 * p + 1] ? n1 : ZSENT);
+      }
+    // stage 2: {S1, P[9..16]}
+    group_sum<FMT, F, 8, 8, R, CC, NV3>(P, rl, cl, Np, X, nmin, S);
+  } else {
+    // one stage: {C, P[1..16]}
+    group_sum<FMT, F, 0, 16, R, CC, NV3>(P, rl, cl, Np, X, nmin, S);
+  }
+
+  // toward-zero write-back into the state (the fp32 value is its top 24 bits)
   uint32_t rare = 0;
 #pragma unroll
   for (int r = 0; r < R; r++)
 #pragma unroll
-    for (int c = 0; c < CC; c++) {
-      uint32_t rr;
-      D[r][c] = cast_normal<F>(S[r][c], nmin[r][c], rr);
-      rare |= rr << (r * CC + c);
+    for (int p = 0; p < CC / 2; p++) {
+      int32_t n0, n1;
+      to_state<F>(S[r][2 * p], nmin[r][2 * p], n0, X[r][2 * p], XMASK);
+      to_state<F>(S[r][2 * p + 1], nmin[r][2 * p + 1], n1, X[r][2 * p + 1], XMASK);
+      Np[r][p] = pack16(n0, n1);
+      // zero (X == 0 exactly when S == 0), or the exponent outside [-126, 127]
+      const bool odd0 = (X[r][2 * p] == 0) || ((uint32_t)(n0 + 127) > 253u);
+      const bool odd1 = (X[r][2 * p + 1] == 0) || ((uint32_t)(n1 + 127) > 253u);
+      rare |= (odd0 ? (1u << (r * CC + 2 * p)) : 0u) | (odd1 ? (1u << (r * CC + 2 * p + 1)) : 0u);
     }
+  dneg0 &= rare;  // every ordinary result is nonzero
+
   if (rare) {
+    // Only the new state is used here: S == 0 left X == 0, and for S != 0
+    // X ^ sgn = (|S| << clz) >> 1 with n = -(exponent of the leading bit).
 #pragma unroll
     for (int r = 0; r < R; r++)
 #pragma unroll
       for (int c = 0; c < CC; c++) {
         const uint32_t bit = 1u << (r * CC + c);
         if (!(rare & bit)) continue;
-        if (S[r][c] != 0) {
-          D[r][c] = cast_out_of_range<F>(S[r][c], nmin[r][c]);
-        } else {
+        const int32_t x0 = X[r][c];
+        const int32_t n0 = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
+        const uint32_t sg = (uint32_t)(x0 >> 31);
+        int32_t n;
+        int32_t x;
+        bool negz = false;
+        if (x0 == 0) {
           // zero-sign rule: -0 only when C and all 16 products are -0
-          bool neg = (c_negzero & bit) != 0;
+          bool neg = (dneg0 & bit) != 0;
           for (int k = 0; k < 16 && neg; k++) {
             const bool zero = P.aN[k][rl + r] == ZSENT || P.bN[k][cl + c] == ZSENT;
-            neg = zero && ((P.aS[k][rl + r] ^ P.bS[k][cl + c]) != 0u);
+            neg = zero && ((P.aS[k][rl + r] ^ P.bS[k][cl + c]) & 0x80000000u) != 0u;
           }
-          D[r][c] = neg ? 0x80000000u : 0u;
+          n = ZSENT;
+          x = neg ? -1 : 0;
+          negz = neg;
+        } else if (n0 <= STATE_NAN + 50) {  // a NaN carried in
+          n = STATE_NAN;
+          x = 0x40000000;
+        } else if (n0 < -127) {  // exponent above 127: overflow to infinity
+          n = STATE_INF;
+          x = (int32_t)(0x40000000u ^ sg);
+        } else {
+          // below 2^-126: truncate onto the subnormal grid 2^-149, i.e.
+          // q = floor(|S| 2^(e_max - F + 149)) = ((X ^ sgn) >> (n - 119))
+          const uint32_t q = shr_u32((uint32_t)x0 ^ sg, (uint32_t)(n0 - 119));
+          if (q == 0) {
+            n = ZSENT;
+            x = (int32_t)sg;
+            negz = sg != 0;
+          } else {
+            n = 126;
+            x = (int32_t)((q << 7) ^ sg);
+          }
         }
+        X[r][c] = x;
+        Np[r][c / 2] = (c & 1) ? pack16(lo16(Np[r][c / 2]), n) : pack16(n, hi16(Np[r][c / 2]));
+        dneg0 = negz ? (dneg0 | bit) : (dneg0 & ~bit);
       }
   }
 
   // special values: NaN anywhere or Inf x 0 -> NaN; Inf of one sign -> that
   // Inf; both signs -> NaN
-  if (panel_special || (c_nan | c_infp | c_infn)) {
+  if (panel_special) {
+    const uint64_t codes = special_codes<R, CC>(&P, rl, cl, c_nan, c_infp, c_infn);
 #pragma unroll
     for (int r = 0; r < R; r++)
 #pragma unroll
       for (int c = 0; c < CC; c++) {
-        const uint32_t bit = 1u << (r * CC + c);
-        bool nan = (c_nan & bit) != 0, ip = (c_infp & bit) != 0, in = (c_infn & bit) != 0;
-        if (panel_special) {
-          for (int k = 0; k < 16; k++) {
-            const int32_t an = P.aN[k][rl + r], bn = P.bN[k][cl + c];
-            if (an == NNAN || bn == NNAN) {
-              nan = true;
-            } else if (an == NINF || bn == NINF) {
-              if (an == ZSENT || bn == ZSENT) nan = true;
-              else if (P.aS[k][rl + r] ^ P.bS[k][cl + c]) in = true;
-              else ip = true;
-            }
-          }
-        }
-        if (nan || (ip && in)) D[r][c] = 0x7FC00000u;
-        else if (ip) D[r][c] = 0x7F800000u;
-        else if (in) D[r][c] = 0xFF800000u;
+        const uint32_t code = (uint32_t)(codes >> (2 * (r * CC + c))) & 3u;
+        if (code == 0u) continue;
+        const int32_t n = code == 1u ? STATE_NAN : STATE_INF;
+        X[r][c] = code == 3u ? (int32_t)0xBFFFFFFFu : 0x40000000;
+        Np[r][c / 2] = (c & 1) ? pack16(lo16(Np[r][c / 2]), n) : pack16(n, hi16(Np[r][c / 2]));
+        dneg0 &= ~(1u << (r * CC + c));
       }
   }
+}
+
+// state of an R x CC block from fp32 C values (row stride ldc), or +0
+template <int R, int CC>
+__device__ __forceinline__ void load_state(const float *C, size_t ldc, bool have_c, uint32_t (&Np)[R][CC / 2],
+                                           int32_t (&X)[R][CC], uint32_t &dneg0) {
+  dneg0 = 0;
+#pragma unroll
+  for (int r = 0; r < R; r++) {
+    uint32_t cv[CC];
+    if (have_c) {
+#pragma unroll
+      for (int q = 0; q < CC / 4; q++) {
+        const uint4 v = reinterpret_cast<const uint4 *>(C + r * ldc)[q];
+        cv[4 * q] = v.x; cv[4 * q + 1] = v.y; cv[4 * q + 2] = v.z; cv[4 * q + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < CC; c++) cv[c] = 0u;
+    }
+    int32_t n[CC];
+#pragma unroll
+    for (int c = 0; c < CC; c++) {
+      bool nz;
+      state_from_fp32(cv[c], n[c], X[r][c], nz);
+      if (nz) dneg0 |= 1u << (r * CC + c);
+    }
+#pragma unroll
+    for (int p = 0; p < CC / 2; p++) Np[r][p] = pack16(n[2 * p], n[2 * p + 1]);
+  }
+}
+
+template <int R, int CC>
+__device__ __forceinline__ void state_to_fp32(const uint32_t (&Np)[R][CC / 2], const int32_t (&X)[R][CC],
+                                              uint32_t (&D)[R][CC]) {
+#pragma unroll
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int c = 0; c < CC; c++)
+      D[r][c] = fp32_from_state((c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]), X[r][c]);
 }
 
 // ---------------------------------------------------------------------------
@@ -280,6 +419,8 @@ __device__ __forceinline__ uint32_t store_a8(Panel<BM, BN> &P, int m, int h, con
     P.aM[8 * h + i][m] = d.m << SH;
     P.aN[8 * h + i][m] = d.n;
     P.aS[8 * h + i][m] = d.s;
+    P.aP[8 * h + i][m] = (int32_t)(d.s | 1u);
+    P.aN2[8 * h + i][m] = pack16(d.n, d.n);
     signs |= (d.s & 1u) << i;
     special |= d.special;
   }
@@ -287,15 +428,19 @@ __device__ __forceinline__ uint32_t store_a8(Panel<BM, BN> &P, int m, int h, con
   return special;
 }
 
-template <int FMT, int BM, int BN>
+// Decode 8 k-consecutive elements of B column n; the column's class (IMAD or
+// ones' complement signs) decides the form of bS.
+template <int FMT, int CC, int NV3, int BM, int BN>
 __device__ __forceinline__ uint32_t store_b8(Panel<BM, BN> &P, int n, int h, const Raw8<FMT> &raw) {
   uint32_t signs = 0, special = 0;
+  const bool pm1 = (n % CC) < NV3;
 #pragma unroll
   for (int i = 0; i < 8; i++) {
     const Dec d = decode<FMT>(raw.get(i));
     P.bM[8 * h + i][n] = d.m;
     P.bN[8 * h + i][n] = d.n;
-    P.bS[8 * h + i][n] = d.s;
+    P.bS[8 * h + i][n] = pm1 ? (d.s | 1u) : d.s;
+    P.bN2[8 * h + i][n] = (int16_t)d.n;
     signs |= (d.s & 1u) << i;
     special |= d.special;
   }
@@ -306,21 +451,21 @@ __device__ __forceinline__ uint32_t store_b8(Panel<BM, BN> &P, int n, int h, con
 // ---------------------------------------------------------------------------
 // GEMM
 // ---------------------------------------------------------------------------
-constexpr int GBM = 64, GBN = 128, GTHREADS = 256;
+constexpr int GBM = 64, GBN = 128, GTHREADS = 256, GR = 4, GCC = 8, GNV3 = 5;
 using GPanel = Panel<GBM, GBN>;
 
 template <int MODEL, int FMT>
-__global__ void __launch_bounds__(GTHREADS) gemm_kernel(const void *__restrict__ A, const void *__restrict__ B,
-                                                        const float *__restrict__ C, float *__restrict__ Dout,
-                                                        uint32_t *__restrict__ fp, int M, int N, int K) {
+__global__ void __launch_bounds__(GTHREADS, 1) gemm_kernel(const void *__restrict__ A, const void *__restrict__ B,
+                                                           const float *__restrict__ C, float *__restrict__ Dout,
+                                                           uint32_t *__restrict__ fp, int M, int N, int K) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   GPanel *panels = reinterpret_cast<GPanel *>(smem_raw);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row0 = blockIdx.y * GBM, col0 = blockIdx.x * GBN;
   // this thread's 4 x 8 outputs
-  const int rl = (warp >> 2) * 32 + (lane >> 2) * 4;
-  const int cl = (warp & 3) * 32 + (lane & 3) * 8;
+  const int rl = (warp >> 2) * 32 + (lane >> 2) * GR;
+  const int cl = (warp & 3) * 32 + (lane & 3) * GCC;
   const bool out_valid = (row0 + rl < M) && (col0 + cl < N);
 
   // loader roles: A row am / half ah (threads < 128); B column bn / half bh
@@ -340,37 +485,29 @@ __global__ void __launch_bounds__(GTHREADS) gemm_kernel(const void *__restrict__
   auto store_chunk = [&](GPanel &P) -> uint32_t {
     uint32_t sp = 0;
     if (a_loader) sp |= store_a8<MODEL, FMT>(P, am, ah, ra);
-    sp |= store_b8<FMT>(P, bn, bh, rb);
+    sp |= store_b8<FMT, GCC, GNV3>(P, bn, bh, rb);
     return sp;
   };
 
-  // accumulator input
-  uint32_t D[4][8];
-#pragma unroll
-  for (int i = 0; i < 4; i++) {
-    if (C != nullptr && out_valid) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(C + (size_t)(row0 + rl + i) * N + col0 + cl);
-      const uint4 a = src[0], b = src[1];
-      D[i][0] = a.x; D[i][1] = a.y; D[i][2] = a.z; D[i][3] = a.w;
-      D[i][4] = b.x; D[i][5] = b.y; D[i][6] = b.z; D[i][7] = b.w;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; j++) D[i][j] = 0u;
-    }
-  }
+  uint32_t Np[GR][GCC / 2];
+  int32_t X[GR][GCC];
+  uint32_t dneg0;
+  load_state<GR, GCC>(C + (size_t)(row0 + rl) * N + col0 + cl, (size_t)N, C != nullptr && out_valid, Np, X, dneg0);
 
   load_chunk(0);
   bool panel_special = __syncthreads_or(store_chunk(panels[0])) != 0;
   for (int j = 0; j < nchunks; j++) {
     if (j + 1 < nchunks) load_chunk(j + 1);
-    mma_chunk<MODEL, FMT, 4, 8>(panels[j & 1], rl, cl, D, panel_special);
+    mma_chunk<MODEL, FMT, GR, GCC, GNV3>(panels[j & 1], rl, cl, Np, X, dneg0, panel_special);
     if (j + 1 < nchunks) panel_special = __syncthreads_or(store_chunk(panels[(j + 1) & 1])) != 0;
   }
 
   // epilogue: store D and the per-16x16-tile xorsum
+  uint32_t D[GR][GCC];
+  state_to_fp32<GR, GCC>(Np, X, D);
   if (out_valid) {
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
+    for (int i = 0; i < GR; i++) {
       uint4 *dst = reinterpret_cast<uint4 *>(Dout + (size_t)(row0 + rl + i) * N + col0 + cl);
       dst[0] = make_uint4(D[i][0], D[i][1], D[i][2], D[i][3]);
       dst[1] = make_uint4(D[i][4], D[i][5], D[i][6], D[i][7]);
@@ -379,9 +516,9 @@ __global__ void __launch_bounds__(GTHREADS) gemm_kernel(const void *__restrict__
   if (fp != nullptr) {
     uint32_t x = 0;
 #pragma unroll
-    for (int i = 0; i < 4; i++)
+    for (int i = 0; i < GR; i++)
 #pragma unroll
-      for (int j = 0; j < 8; j++) x ^= D[i][j];
+      for (int j = 0; j < GCC; j++) x ^= D[i][j];
     // the 8 lanes sharing a 16x16 tile differ in lane bits 0, 2, 3
     x ^= __shfl_xor_sync(0xFFFFFFFFu, x, 1);
     x ^= __shfl_xor_sync(0xFFFFFFFFu, x, 4);
@@ -396,7 +533,7 @@ __global__ void __launch_bounds__(GTHREADS) gemm_kernel(const void *__restrict__
 // ---------------------------------------------------------------------------
 // independent tiles: one warp per 16x16x16 tile, each lane 2 x 4 outputs
 // ---------------------------------------------------------------------------
-constexpr int TWARPS = 8;
+constexpr int TWARPS = 8, TR = 2, TCC = 4, TNV3 = 2;
 using TPanel = Panel<16, 16>;
 
 template <int MODEL, int FMT>
@@ -406,29 +543,25 @@ __global__ void __launch_bounds__(TWARPS * 32) tiles_kernel(const void *__restri
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   TPanel &P = reinterpret_cast<TPanel *>(smem_raw)[warp];
-  const int rl = (lane >> 2) * 2, cl = (lane & 3) * 4;
+  const int rl = (lane >> 2) * TR, cl = (lane & 3) * TCC;
   const int lm = lane & 15, lh = lane >> 4;
   for (size_t t = (size_t)blockIdx.x * TWARPS + warp; t < ntiles; t += (size_t)gridDim.x * TWARPS) {
     const Raw8<FMT> ra = load_row8<FMT>(A, t * 256 + lm * 16 + 8 * lh, true);
     const Raw8<FMT> rb = load_col8<FMT>(B, t * 256 + (8 * lh) * 16 + lm, 16, true);
-    uint32_t D[2][4];
-#pragma unroll
-    for (int i = 0; i < 2; i++) {
-      if (C != nullptr) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(C + t * 256 + (rl + i) * 16 + cl);
-        D[i][0] = v.x; D[i][1] = v.y; D[i][2] = v.z; D[i][3] = v.w;
-      } else {
-        D[i][0] = D[i][1] = D[i][2] = D[i][3] = 0u;
-      }
-    }
+    uint32_t Np[TR][TCC / 2];
+    int32_t X[TR][TCC];
+    uint32_t dneg0;
+    load_state<TR, TCC>(C + t * 256 + rl * 16 + cl, 16, C != nullptr, Np, X, dneg0);
     __syncwarp();  // the previous tile's reads of P are done
     uint32_t sp = store_a8<MODEL, FMT>(P, lm, lh, ra);
-    sp |= store_b8<FMT>(P, lm, lh, rb);
+    sp |= store_b8<FMT, TCC, TNV3>(P, lm, lh, rb);
     const bool panel_special = __any_sync(0xFFFFFFFFu, sp != 0);
     __syncwarp();
-    mma_chunk<MODEL, FMT, 2, 4>(P, rl, cl, D, panel_special);
+    mma_chunk<MODEL, FMT, TR, TCC, TNV3>(P, rl, cl, Np, X, dneg0, panel_special);
+    uint32_t D[TR][TCC];
+    state_to_fp32<TR, TCC>(Np, X, D);
 #pragma unroll
-    for (int i = 0; i < 2; i++)
+    for (int i = 0; i < TR; i++)
       *reinterpret_cast<uint4 *>(Dout + t * 256 + (rl + i) * 16 + cl) = make_uint4(D[i][0], D[i][1], D[i][2], D[i][3]);
   }
 }

@@ -47,7 +47,28 @@ SMS, LANES_PER_SM, MAX_SM_MHZ = 148, 128, 1965.0
 ALU_PEAK_TOPS = SMS * LANES_PER_SM * MAX_SM_MHZ * 1e6 / 1e12
 H2D_BYTES = M * K * 2 + K * N * 2 + M * N * 4
 D2H_BYTES = M * N * 4 + (M // 16) * (N // 16) * 4
+ALGO_BYTES = H2D_BYTES + D2H_BYTES  # A, B, C read and D, fingerprints written once
 WORKLOAD = "gemm M=N=K=4096, Ampere FP16 model, fp32 C=0 and D, fused per-16x16-tile xorsum"
+# DRAM bytes per launch of the GEMM kernel (dram__bytes_read.sum + dram__bytes_write.sum)
+# from one ncu capture (profiles/gemm_ampere_fp16_4096_ncu_full.md), valid only
+# for the kernel sources it was taken on, identified by their hash.
+TRAFFIC_CAPTURE = {"source_sha16": "459e36c031f5fe18", "bytes": 231_652_352}
+KERNEL_SOURCES = ("bit_exact_tensor_b200/csrc/mmaemu.cu", "bit_exact_tensor_b200/csrc/mmaemu_core.cuh",
+                  "include/mmaemu.h")
+
+
+def kernel_source_sha16() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    return TRAFFIC_CAPTURE["bytes"] if kernel_source_sha16() == TRAFFIC_CAPTURE["source_sha16"] else None
 
 
 def parse():
@@ -197,6 +218,27 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# multi-rank host logic
+# ---------------------------------------------------------------------------
+def reduce_max(x: float, dist=None, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a process
+    group).  Works with NCCL (device tensor) and gloo (CPU tensor)."""
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(step_ms_max: float, world: int) -> float:
+    """Whole-job emulated MACs/s: every rank runs one full problem per step
+    (weak scaling), timed by the slowest rank."""
+    return MACS_PER_STEP * world / (step_ms_max / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
 def run_gpu(args):
@@ -222,11 +264,7 @@ def run_gpu(args):
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, dist, dev)
 
     A_np, B_np, C_np = wl.config3(seed=3 + 1000 * rank)
     A = torch.from_numpy(A_np.view(np.int16)).to(dev)
@@ -289,7 +327,7 @@ def run_gpu(args):
     barrier()
 
     if rank == 0:
-        value = MACS_PER_STEP * world / (total_ms / 1e3 / args.steps)
+        value = aggregate_value(total_ms / args.steps, world)
         achieved = OPS_PER_MAC * MACS_PER_STEP / (kern_ms / 1e3) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -300,7 +338,8 @@ def run_gpu(args):
                        "input_format": "fp16", "global_batch": world, "parallelism": f"independent x{world}",
                        "l2": "inputs larger than L2 (192 MiB working set per GPU)"},
             "roofline": {"bound": "alu", "achieved": achieved, "peak": ALU_PEAK_TOPS, "unit": "Tops/s",
-                         "frac": achieved / ALU_PEAK_TOPS, "traffic": None,
+                         "frac": achieved / ALU_PEAK_TOPS, "traffic": measured_traffic(),
+                         "traffic_unit": "bytes per launch", "algorithmic_bytes": ALGO_BYTES,
                          "kernel": "gemm_kernel<ampere,fp16>", "ops_per_mac": OPS_PER_MAC,
                          "peak_basis": "148 SM x 128 lanes x 1965 MHz issue ceiling (derived)"},
             "clocks": clocks,

@@ -43,6 +43,11 @@ struct __align__(16) Panel {
   uint16_t sb16[BN];     // bit k = sign of b[k][n]
 };
 
+#ifndef MMAEMU_KUNROLL
+#define MMAEMU_KUNROLL 1
+#endif
+constexpr int KUNROLL = MMAEMU_KUNROLL;
+
 template <int R, typename T>
 __device__ __forceinline__ void lds_vec(const T *p, T (&v)[R]) {
   static_assert(sizeof(T) == 4, "32-bit elements");
@@ -75,7 +80,7 @@ __device__ __forceinline__ void group_sum(const Panel<BM, BN> &P, int rl, int cl
   for (int r = 0; r < R; r++)
 #pragma unroll
     for (int p = 0; p < CC / 2; p++) nm2[r][p] = Np[r][p];
-#pragma unroll 1
+#pragma unroll KUNROLL
   for (int k = K0; k < K0 + KN; k++) {
     uint32_t an2[R], bn2[CC / 2];
     lds_vec<R>(&P.aN2[k][rl], an2);
@@ -103,7 +108,7 @@ __device__ __forceinline__ void group_sum(const Panel<BM, BN> &P, int rl, int cl
       const int32_t nc = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
       S[r][c] = shr_s32(X[r][c], (uint32_t)(nc - nmin[r][c] + CSH)) - (X[r][c] >> 31);
     }
-#pragma unroll 1
+#pragma unroll KUNROLL
   for (int k = K0; k < K0 + KN; k++) {
     uint32_t am[R], as[R], bm[CC], bs[CC];
     int32_t an[R], ap[R], bn[CC];
@@ -114,10 +119,11 @@ __device__ __forceinline__ void group_sum(const Panel<BM, BN> &P, int rl, int cl
     lds_vec<CC>(&P.bM[k][cl], bm);
     lds_vec<CC>(&P.bN[k][cl], bn);
     lds_vec<CC>(&P.bS[k][cl], bs);
+    // column-outer order: measured faster (operand reuse across rows)
 #pragma unroll
-    for (int r = 0; r < R; r++)
+    for (int c = 0; c < CC; c++)
 #pragma unroll
-      for (int c = 0; c < CC; c++) {
+      for (int r = 0; r < R; r++) {
         const uint32_t T = shr_u32(am[r] * bm[c], (uint32_t)(an[r] + bn[c] - nmin[r][c]));
         if (c < NV3) {
           S[r][c] += (int32_t)T * (ap[r] * (int32_t)bs[c]);
@@ -451,11 +457,19 @@ __device__ __forceinline__ uint32_t store_b8(Panel<BM, BN> &P, int n, int h, con
 // ---------------------------------------------------------------------------
 // GEMM
 // ---------------------------------------------------------------------------
-constexpr int GBM = 64, GBN = 128, GTHREADS = 256, GR = 4, GCC = 8, GNV3 = 5;
+// Tuning knobs (compile-time): IMAD-sign columns per thread, resident
+// blocks per SM, and the unroll of the k loops.
+#ifndef MMAEMU_GNV3
+#define MMAEMU_GNV3 8
+#endif
+#ifndef MMAEMU_GMINB
+#define MMAEMU_GMINB 2
+#endif
+constexpr int GBM = 64, GBN = 128, GTHREADS = 256, GR = 4, GCC = 8, GNV3 = MMAEMU_GNV3;
 using GPanel = Panel<GBM, GBN>;
 
 template <int MODEL, int FMT>
-__global__ void __launch_bounds__(GTHREADS, 1) gemm_kernel(const void *__restrict__ A, const void *__restrict__ B,
+__global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const void *__restrict__ A, const void *__restrict__ B,
                                                            const float *__restrict__ C, float *__restrict__ Dout,
                                                            uint32_t *__restrict__ fp, int M, int N, int K) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -533,7 +547,7 @@ __global__ void __launch_bounds__(GTHREADS, 1) gemm_kernel(const void *__restric
 // ---------------------------------------------------------------------------
 // independent tiles: one warp per 16x16x16 tile, each lane 2 x 4 outputs
 // ---------------------------------------------------------------------------
-constexpr int TWARPS = 8, TR = 2, TCC = 4, TNV3 = 2;
+constexpr int TWARPS = 8, TR = 2, TCC = 4, TNV3 = 4;
 using TPanel = Panel<16, 16>;
 
 template <int MODEL, int FMT>

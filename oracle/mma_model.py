@@ -37,6 +37,17 @@ Everything is done with Python integers, so no step can round by accident.
 Where the pages leave a point open, the reading taken is stated next to the
 code (readings R1..R12, listed with the same numbers in the design notes).
 
+Pins: the worked example, the five target-test outcomes, the Algorithm 4
+neutral-subgroup structure, Algorithm 10 and the -133 threshold fix
+decode, product_term, group_sum, normalise, cast_rz and mma_element against
+the pages; an exact-rational restatement and exhaustive toy formats fix
+them against the rules as read.  Parity unpinned (the pages are silent, so
+only the stated reading is fixed, not hardware behaviour): the internal width
+used for BF16 and E4M3 (R3), truncation at the stage hand-over (R4), zero
+terms left out of the max exponent (R5), subnormal fp32 C (R8), NaN/Inf
+handling and gradual underflow of results (R9), and the sign of zero
+results (R12).
+
 Conventions
 -----------
 * A decoded finite value is (s, e, m): value = (-1)^s * m * 2^(e - p), with

@@ -52,9 +52,57 @@ WORKLOAD = "gemm M=N=K=4096, Ampere FP16 model, fp32 C=0 and D, fused per-16x16-
 # DRAM bytes per launch of the GEMM kernel (dram__bytes_read.sum + dram__bytes_write.sum)
 # from one ncu capture (profiles/gemm_ampere_fp16_4096_ncu_full.md), valid only
 # for the kernel sources it was taken on, identified by their hash.
-TRAFFIC_CAPTURE = {"source_sha16": "459e36c031f5fe18", "bytes": 231_652_352}
+TRAFFIC_CAPTURE = {"source_sha16": "323bd3c1a42c7bb3", "bytes": 200_515_072}
 KERNEL_SOURCES = ("bit_exact_tensor_b200/csrc/mmaemu.cu", "bit_exact_tensor_b200/csrc/mmaemu_core.cuh",
                   "include/mmaemu.h")
+
+
+HBM_PEAK_GBS = 6557.4  # measured copy bandwidth on this machine's B200s (MEASURED_PEAKS.json)
+DEFAULT_WORKLOAD = "gemm-ampere-fp16-4096"
+PAIRS = (("ampere", "fp16"), ("ampere", "bf16"), ("hopper", "fp16"), ("hopper", "bf16"), ("hopper", "e4m3"))
+WORKLOAD_NAMES = ({DEFAULT_WORKLOAD, "gemm-hopper-bf16-4096", "gemm-hopper-bf16-4096-wide",
+                   "gemm-hopper-e4m3-8192x4096x14336", "tiles-ampere-fp16-4096"}
+                  | {f"tiles-{m}-{f}-100k" for m, f in PAIRS})
+
+
+def workload_spec(name: str) -> dict:
+    """Inputs and byte/MAC counts of a named workload (the configurations of
+    the Hawkeye workloads: random 16x16x16 tiles and large GEMMs)."""
+    from bit_exact_tensor_b200 import workloads as wl
+
+    def gemm(model, fmt, make, M_, N_, K_, desc):
+        eb = 1 if fmt == "e4m3" else 2
+        return {"kind": "gemm", "model": model, "fmt": fmt, "make": make, "macs": M_ * N_ * K_, "desc": desc,
+                "h2d": (M_ * K_ + K_ * N_) * eb + M_ * N_ * 4, "d2h": M_ * N_ * 4 + (M_ // 16) * (N_ // 16) * 4,
+                "l2": "inputs larger than L2"}
+
+    def tiles(model, fmt, make, nt, desc):
+        eb = 1 if fmt == "e4m3" else 2
+        return {"kind": "tiles", "model": model, "fmt": fmt, "make": make, "macs": nt * 4096, "desc": desc,
+                "h2d": nt * 256 * (2 * eb + 4), "d2h": nt * 1024,
+                "l2": "inputs larger than L2" if nt * 256 * (2 * eb + 8) > 126e6 else "fits in L2"}
+
+    if name == DEFAULT_WORKLOAD:
+        return gemm("ampere", "fp16", lambda r: wl.config3(seed=3 + 1000 * r), M, N, K, WORKLOAD)
+    if name == "gemm-hopper-bf16-4096":
+        return gemm("hopper", "bf16", lambda r: wl.config4(seed=4 + 1000 * r), 4096, 4096, 4096,
+                    "gemm M=N=K=4096, Hopper BF16 model, log2|x| ~ U[-60, 60], fused per-tile xorsum")
+    if name == "gemm-hopper-bf16-4096-wide":
+        return gemm("hopper", "bf16", lambda r: wl.config4(seed=4 + 1000 * r, wide=True), 4096, 4096, 4096,
+                    "gemm M=N=K=4096, Hopper BF16 model, log2|x| ~ U[-126, 127], fused per-tile xorsum")
+    if name == "gemm-hopper-e4m3-8192x4096x14336":
+        return gemm("hopper", "e4m3", lambda r: wl.config5(seed=5 + 1000 * r), 8192, 14336, 4096,
+                    "gemm M=8192 K=4096 N=14336, Hopper E4M3 model, N(0,1)/sqrt(K), fused per-tile xorsum")
+    if name == "tiles-ampere-fp16-4096":
+        return tiles("ampere", "fp16", lambda r: wl.config1(seed=0 + 1000 * r), 4096,
+                     "4,096 tiles 16x16x16, Ampere FP16 model, 10% subnormal entries")
+    for m, f in PAIRS:
+        if name == f"tiles-{m}-{f}-100k":
+            def make(r, f=f):
+                A_, B_, C_, _ = wl.config2(f, seed=1 + 1000 * r)
+                return A_, B_, C_
+            return tiles(m, f, make, 100_000, f"100,000 random + adversarial tiles, {m.capitalize()} {f.upper()} model")
+    raise ValueError(name)
 
 
 def kernel_source_sha16() -> str:
@@ -79,6 +127,8 @@ def parse():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOAD_NAMES),
+                    help="which workload to time (default: the headline 4096^3 FP16-Ampere GEMM)")
     return ap.parse_args()
 
 
@@ -232,10 +282,10 @@ def reduce_max(x: float, dist=None, device=None) -> float:
     return float(t.item())
 
 
-def aggregate_value(step_ms_max: float, world: int) -> float:
+def aggregate_value(step_ms_max: float, world: int, macs_per_step: int = MACS_PER_STEP) -> float:
     """Whole-job emulated MACs/s: every rank runs one full problem per step
     (weak scaling), timed by the slowest rank."""
-    return MACS_PER_STEP * world / (step_ms_max / 1e3)
+    return macs_per_step * world / (step_ms_max / 1e3)
 
 
 # ---------------------------------------------------------------------------
@@ -266,16 +316,23 @@ def run_gpu(args):
     def max_over_ranks(x: float) -> float:
         return reduce_max(x, dist, dev)
 
-    A_np, B_np, C_np = wl.config3(seed=3 + 1000 * rank)
-    A = torch.from_numpy(A_np.view(np.int16)).to(dev)
-    B = torch.from_numpy(B_np.view(np.int16)).to(dev)
+    spec = workload_spec(args.workload)
+    A_np, B_np, C_np = spec["make"](rank)
+    A = torch.from_numpy(A_np.view(np.uint8 if spec["fmt"] == "e4m3" else np.int16)).to(dev)
+    B = torch.from_numpy(B_np.view(np.uint8 if spec["fmt"] == "e4m3" else np.int16)).to(dev)
     C = torch.from_numpy(C_np.view(np.int32)).to(dev)
-    D = torch.empty((M, N), dtype=torch.float32, device=dev)
-    fp = torch.empty(((M // 16) * (N // 16),), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    if spec["kind"] == "gemm":
+        D = torch.empty(C.shape, dtype=torch.float32, device=dev)
+        fp = torch.empty(((C.shape[0] // 16) * (C.shape[1] // 16),), dtype=torch.int32, device=dev)
 
-    def step():
-        mmaemu.gemm("ampere", "fp16", A, B, C, out=D, fp_out=fp)
+        def step():
+            mmaemu.gemm(spec["model"], spec["fmt"], A, B, C, out=D, fp_out=fp)
+    else:
+        D = torch.empty(C.shape, dtype=torch.float32, device=dev)
+
+        def step():
+            mmaemu.tiles(spec["model"], spec["fmt"], A, B, C, out=D)
 
     for _ in range(args.warmup):
         step()
@@ -310,44 +367,63 @@ def run_gpu(args):
     kern_ms = max_over_ranks(sum(per_ms) / len(per_ms))
 
     # end to end through the public API from pinned host buffers
-    A_h = torch.from_numpy(A_np.view(np.int16)).pin_memory()
-    B_h = torch.from_numpy(B_np.view(np.int16)).pin_memory()
+    A_h = torch.from_numpy(A_np.view(np.uint8 if spec["fmt"] == "e4m3" else np.int16)).pin_memory()
+    B_h = torch.from_numpy(B_np.view(np.uint8 if spec["fmt"] == "e4m3" else np.int16)).pin_memory()
     C_h = torch.from_numpy(C_np.view(np.int32)).pin_memory()
-    mmaemu.gemm_host("ampere", "fp16", A_h, B_h, C_h, device=dev)  # warm-up
+
+    def e2e_step():
+        if spec["kind"] == "gemm":
+            return mmaemu.gemm_host(spec["model"], spec["fmt"], A_h, B_h, C_h, device=dev)
+        Ad, Bd, Cd = (t.to(dev, non_blocking=True) for t in (A_h, B_h, C_h))
+        Dh = torch.empty(C_h.shape, dtype=torch.float32, pin_memory=True)
+        Dh.copy_(mmaemu.tiles(spec["model"], spec["fmt"], Ad, Bd, Cd), non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+        return Dh, None
+
+    e2e_step()  # warm-up
     barrier()
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.e2e_steps):
-        D_h, fp_h = mmaemu.gemm_host("ampere", "fp16", A_h, B_h, C_h, device=dev)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps)
     barrier()
 
     if rank == 0:
-        value = aggregate_value(total_ms / args.steps, world)
-        achieved = OPS_PER_MAC * MACS_PER_STEP / (kern_ms / 1e3) / 1e12
+        macs = spec["macs"]
+        value = aggregate_value(total_ms / args.steps, world, macs)
+        achieved = OPS_PER_MAC * macs / (kern_ms / 1e3) / 1e12
+        h2d, d2h = spec["h2d"], spec["d2h"]
+        roof = {"bound": "alu", "achieved": achieved, "peak": ALU_PEAK_TOPS, "unit": "Tops/s",
+                "frac": achieved / ALU_PEAK_TOPS,
+                "traffic": measured_traffic() if args.workload == DEFAULT_WORKLOAD else None,
+                "traffic_unit": "bytes per launch", "algorithmic_bytes": h2d + d2h,
+                "kernel": f"{spec['kind']}_kernel<{spec['model']},{spec['fmt']}>", "ops_per_mac": OPS_PER_MAC,
+                "peak_basis": "148 SM x 128 lanes x 1965 MHz issue ceiling (derived)"}
+        if spec["kind"] == "tiles":  # mixed bound: also report HBM against the measured copy bandwidth
+            hbm = (h2d + d2h) / (kern_ms / 1e3) / 1e9
+            roof.update({"hbm_achieved_gbs": hbm, "hbm_peak_gbs": HBM_PEAK_GBS, "hbm_frac": hbm / HBM_PEAK_GBS})
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": METRIC if args.workload == DEFAULT_WORKLOAD else f"emulated MACs/s, {spec['desc']}",
+            "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": value / PAGES_MACS_PER_S, "dtype": "int32",
-            "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K, "emulated_arch": "ampere",
-                       "input_format": "fp16", "global_batch": world, "parallelism": f"independent x{world}",
-                       "l2": "inputs larger than L2 (192 MiB working set per GPU)"},
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": ALU_PEAK_TOPS, "unit": "Tops/s",
-                         "frac": achieved / ALU_PEAK_TOPS, "traffic": measured_traffic(),
-                         "traffic_unit": "bytes per launch", "algorithmic_bytes": ALGO_BYTES,
-                         "kernel": "gemm_kernel<ampere,fp16>", "ops_per_mac": OPS_PER_MAC,
-                         "peak_basis": "148 SM x 128 lanes x 1965 MHz issue ceiling (derived)"},
+            "scaling": "weak",
+            "vs_baseline": value / PAGES_MACS_PER_S if args.workload == DEFAULT_WORKLOAD else None,
+            "dtype": "int32", "data": "synthetic",
+            "config": {"workload": spec["desc"], "name": args.workload, "emulated_arch": spec["model"],
+                       "input_format": spec["fmt"], "global_batch": world,
+                       "parallelism": f"independent x{world}", "l2": spec["l2"]},
+            "roofline": roof,
             "clocks": clocks,
-            "e2e": {"value": MACS_PER_STEP * world / (e2e_ms / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": H2D_BYTES, "d2h_bytes_per_step": D2H_BYTES},
+            "e2e": {"value": macs * world / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.workload == DEFAULT_WORKLOAD:
             line["cpu_baseline"] = cpu_baseline(inputs=(A_np, B_np, C_np))
         print(json.dumps(line), flush=True)
     if dist is not None:

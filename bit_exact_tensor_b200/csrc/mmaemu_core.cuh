@@ -17,13 +17,12 @@
 //    operands pre-scaled at decode time;
 //  * truncating alignment is a logical right shift of the magnitude by
 //    delta = n_a + n_b - nmin (the PTX shift gives 0 for delta >= 32);
-//  * signs are applied either by an IMAD with sigma_a * sigma_b (+-1), or in
-//    ones' complement (T ^ sgn, sgn = 0 or all ones) with the number of
-//    negative products added back once per group:
-//        sum_k (-1)^s_k T_k  =  sum_k (T_k ^ sgn_k)  +  #{k : s_k = 1};
+//  * a product's sign is applied by an IMAD with sigma_a * sigma_b (+-1), so
+//    the group sum is an exact two's complement integer;
 //  * because ~x shifted arithmetically equals ~(x shifted logically), a carried
 //    term held in ones' complement (the stage-1 result, or C) is aligned with
-//    one arithmetic shift.
+//    one arithmetic shift and turned exact by adding its sign bit:
+//    ~(M >> d) + 1 = -(M >> d).
 //
 // Accumulator state between K chunks: (n, X).  X holds the value's magnitude
 // left-aligned with its leading bit at bit 30, in ones' complement for a

@@ -66,13 +66,11 @@ __device__ __forceinline__ void lds_vec(const T *p, T (&v)[R]) {
   }
 }
 
-// One accumulation group over k in [K0, K0 + KN) with a carried term given by
-// the state (Np, X): returns S (exact signed sum of the aligned terms) and
-// nmin (= -e_max) for every output.
-template <int FMT, int F, int K0, int KN, int R, int CC, int BM, int BN>
-__device__ __forceinline__ void group_sum(const Panel<BM, BN> &P, int rl, int cl, const uint32_t (&Np)[R][CC / 2],
-                                          const int32_t (&X)[R][CC], int32_t (&nmin)[R][CC], int32_t (&S)[R][CC]) {
-  // pass 1: the group's max exponent, two outputs per packed instruction
+// Pass 1 of a group over k in [K0, K0 + KN): nmin (= -e_max) of every output,
+// starting from the carried terms' negated exponents Np (packed pairs).
+template <int FMT, int K0, int KN, int R, int CC, int BM, int BN>
+__device__ __forceinline__ void group_max(const Panel<BM, BN> &P, int rl, int cl, const uint32_t (&Np)[R][CC / 2],
+                                          int32_t (&nmin)[R][CC]) {
   uint32_t nm2[R][CC / 2];
 #pragma unroll
   for (int r = 0; r < R; r++)
@@ -97,16 +95,13 @@ __device__ __forceinline__ void group_sum(const Panel<BM, BN> &P, int rl, int cl
       nmin[r][2 * p] = lo16(v);
       nmin[r][2 * p + 1] = hi16(v);
     }
-  // pass 2: the carried term, then each product aligned (truncated) and added
-  constexpr int CSH = 30 - F;  // the state's significand sits at bits 30..7
-#pragma unroll
-  for (int r = 0; r < R; r++)
-#pragma unroll
-    for (int c = 0; c < CC; c++) {
-      const int32_t nc = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
-      // ones' complement -> exact: ~(M >> d) + 1 = -(M >> d)
-      S[r][c] = shr_s32(X[r][c], (uint32_t)(nc - nmin[r][c] + CSH)) + (int32_t)((uint32_t)X[r][c] >> 31);
-    }
+}
+
+// Pass 2 of a group: add every product's aligned (truncated) magnitude, with
+// its sign, to S (which already holds the carried term's contribution).
+template <int K0, int KN, int R, int CC, int BM, int BN>
+__device__ __forceinline__ void group_products(const Panel<BM, BN> &P, int rl, int cl, const int32_t (&nmin)[R][CC],
+                                               int32_t (&S)[R][CC]) {
 #pragma unroll KUNROLL
   for (int k = K0; k < K0 + KN; k++) {
     uint32_t am[R], bm[CC];
@@ -126,6 +121,24 @@ __device__ __forceinline__ void group_sum(const Panel<BM, BN> &P, int rl, int cl
         S[r][c] += (int32_t)T * (ap[r] * bp[c]);
       }
   }
+}
+
+// One accumulation group with a carried term in the state form (Np, X):
+// returns S (exact signed sum of the aligned terms) and nmin (= -e_max).
+template <int FMT, int F, int K0, int KN, int R, int CC, int BM, int BN>
+__device__ __forceinline__ void group_sum(const Panel<BM, BN> &P, int rl, int cl, const uint32_t (&Np)[R][CC / 2],
+                                          const int32_t (&X)[R][CC], int32_t (&nmin)[R][CC], int32_t (&S)[R][CC]) {
+  group_max<FMT, K0, KN, R, CC>(P, rl, cl, Np, nmin);
+  constexpr int CSH = 30 - F;  // the state's significand sits at bits 30..7
+#pragma unroll
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int c = 0; c < CC; c++) {
+      const int32_t nc = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
+      // ones' complement -> exact: ~(M >> d) + 1 = -(M >> d)
+      S[r][c] = shr_s32(X[r][c], (uint32_t)(nc - nmin[r][c] + CSH)) + (int32_t)((uint32_t)X[r][c] >> 31);
+    }
+  group_products<K0, KN, R, CC>(P, rl, cl, nmin, S);
 }
 
 // normalise a sum to the state form: X with its leading bit at bit 30 (in
@@ -336,6 +349,218 @@ __device__ __forceinline__ void mma_chunk(const PanelT &P, int rl, int cl, uint3
   }
 }
 
+// ---------------------------------------------------------------------------
+// Float-assisted chunk (FP16 and E4M3 inputs).  The accumulator state is the
+// fp32 value D itself (plus n = -e(D) in packed pairs), and the steps around
+// the integer group sums run on the conversion and FMA units:
+//  * a carried fp32 value c contributes trunc(c 2^(F - e_max)): one exact
+//    multiply by a power of two and one toward-zero conversion to int;
+//  * cvt.rz.f32.s32(S) is S truncated to 24 significant bits with its sign
+//    and exponent -- the Ampere stage hand-over (W = 24) and the fp32
+//    write-back, whose result is that float with (e_max - F) added to its
+//    exponent field.
+// It is exact while every power of two it forms is a normal float, which
+// holds for FP16/E4M3 products and fp32 accumulators of magnitude >= 2^-60
+// (or zero): after a chunk a nonzero D is at least 2^-52 or the incoming C.  Threads whose
+// state leaves that range (Inf/NaN, overflow, tiny nonzero C) switch to the
+// integer path for good.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float i2f_rz(int32_t s) {
+  float f;
+  asm("cvt.rz.f32.s32 %0, %1;" : "=f"(f) : "r"(s));
+  return f;
+}
+__device__ __forceinline__ int32_t f2i_rz(float f) {  // NaN gives 0
+  int32_t r;
+  asm("cvt.rzi.s32.f32 %0, %1;" : "=r"(r) : "f"(f));
+  return r;
+}
+__device__ __forceinline__ int32_t exp_field(float f) {
+  uint32_t r;
+  asm("bfe.u32 %0, %1, 23, 8;" : "=r"(r) : "r"(__float_as_uint(f)));
+  return (int32_t)r;
+}
+// 2^k as a float for k in [-126, 127] (one IMAD)
+__device__ __forceinline__ float pow2f(int32_t k) { return __uint_as_float((uint32_t)k * 0x800000u + 0x3F800000u); }
+
+// accumulators of magnitude below 2^-60 are left to the integer path
+constexpr int FAST_NMAX = 60;
+// BF16 products and sums reach exponents far outside the float range
+template <int FMT> constexpr bool kFloatAssisted = FMT != FMT_BF16;
+
+template <int MODEL, int FMT, int R, int CC, int BM, int BN>
+__device__ __forceinline__ void mma_chunk_fast(const Panel<BM, BN> &P, int rl, int cl, uint32_t (&Np)[R][CC / 2],
+                                               uint32_t (&V)[R][CC], uint32_t &dneg0, bool panel_special,
+                                               bool &to_integer) {
+  constexpr int F = ModelT<MODEL>::F;
+  static_assert(FMT != FMT_BF16, "BF16 exponents leave the float range");
+  int32_t S[R][CC], nmin[R][CC];
+  constexpr int KN1 = MODEL == MODEL_AMPERE ? 8 : 16;
+  // first (or only) group: carried D plus products
+  group_max<FMT, 0, KN1, R, CC>(P, rl, cl, Np, nmin);
+#pragma unroll
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int c = 0; c < CC; c++) S[r][c] = f2i_rz(__uint_as_float(V[r][c]) * pow2f(F + nmin[r][c]));
+  group_products<0, KN1, R, CC>(P, rl, cl, nmin, S);
+  if constexpr (MODEL == MODEL_AMPERE) {
+    // hand-over: the stage-1 sum truncated to 24 bits, carried as
+    // g1 = S1_24 2^(-30 - nmin1) so that only nmin2 is needed next
+    float g1[R][CC];
+#pragma unroll
+    for (int r = 0; r < R; r++)
+#pragma unroll
+      for (int p = 0; p < CC / 2; p++) {
+        int32_t n1[2];
+#pragma unroll
+        for (int q = 0; q < 2; q++) {
+          const int c = 2 * p + q;
+          const float f1 = i2f_rz(S[r][c]);
+          n1[q] = S[r][c] ? nmin[r][c] + (F + 127) - exp_field(f1) : ZSENT;
+          g1[r][c] = f1 * pow2f(-30 - nmin[r][c]);
+        }
+        Np[r][p] = pack16(n1[0], n1[1]);
+      }
+    group_max<FMT, 8, 8, R, CC>(P, rl, cl, Np, nmin);
+#pragma unroll
+    for (int r = 0; r < R; r++)
+#pragma unroll
+      for (int c = 0; c < CC; c++) S[r][c] = f2i_rz(g1[r][c] * pow2f(nmin[r][c] + 30));
+    group_products<8, 8, R, CC>(P, rl, cl, nmin, S);
+  }
+
+  // write-back: D = cvt.rz(S) with e_max - F added to its exponent field
+  bool any_rare = false;
+#pragma unroll
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int p = 0; p < CC / 2; p++) {
+      int32_t nn[2];
+#pragma unroll
+      for (int q = 0; q < 2; q++) {
+        const int c = 2 * p + q;
+        const float f2 = i2f_rz(S[r][c]);
+        nn[q] = nmin[r][c] + (F + 127) - exp_field(f2);
+        V[r][c] = __float_as_uint(f2) - (uint32_t)(nmin[r][c] + F) * 0x800000u;
+        any_rare = any_rare || S[r][c] == 0 || (uint32_t)(nn[q] + 127) > 253u;
+      }
+      Np[r][p] = pack16(nn[0], nn[1]);
+    }
+  uint32_t rare = 0;
+  if (any_rare) {
+#pragma unroll
+    for (int r = 0; r < R; r++)
+#pragma unroll
+      for (int c = 0; c < CC; c++) {
+        const int32_t n0 = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
+        if (!(S[r][c] == 0 || (uint32_t)(n0 + 127) > 253u)) continue;
+        const uint32_t bit = 1u << (r * CC + c);
+        rare |= bit;
+        const int32_t sv = S[r][c];
+        const uint32_t sign = (uint32_t)sv & 0x80000000u;
+        int32_t n;
+        uint32_t d;
+        bool negz = false;
+        if (sv == 0) {
+          // zero-sign rule: -0 only when C and all 16 products are -0
+          bool neg = (dneg0 & bit) != 0;
+          for (int k = 0; k < 16 && neg; k++) {
+            const bool zero = zero_a(P, k, rl + r) || zero_b(P, k, cl + c);
+            neg = zero && (P.aP[k][rl + r] ^ P.bP[k][cl + c]) < 0;
+          }
+          n = ZSENT;
+          d = neg ? 0x80000000u : 0u;
+          negz = neg;
+        } else if (n0 < -127) {  // overflow: infinity, and the integer path from now on
+          n = STATE_INF;
+          d = sign | 0x7F800000u;
+          to_integer = true;
+        } else {  // below 2^-126: truncated onto the subnormal grid 2^-149
+          const uint32_t mag = (uint32_t)(sv < 0 ? -sv : sv);
+          const int sh = -nmin[r][c] - F + 149;
+          const uint32_t q = sh >= 0 ? shl_u32(mag, (uint32_t)sh) : shr_u32(mag, (uint32_t)(-sh));
+          n = q ? 126 : ZSENT;
+          d = sign | q;
+          negz = q == 0 && sign != 0;
+          to_integer = true;  // tiny accumulators are the integer path's
+        }
+        V[r][c] = d;
+        Np[r][c / 2] = (c & 1) ? pack16(lo16(Np[r][c / 2]), n) : pack16(n, hi16(Np[r][c / 2]));
+        dneg0 = negz ? (dneg0 | bit) : (dneg0 & ~bit);
+      }
+  }
+  dneg0 &= rare;
+
+  // Inf/NaN operands (the incoming values are finite on this path)
+  if (panel_special) {
+    const uint64_t codes = special_codes<R, CC>(P, rl, cl, 0u, 0u, 0u);
+#pragma unroll
+    for (int r = 0; r < R; r++)
+#pragma unroll
+      for (int c = 0; c < CC; c++) {
+        const uint32_t code = (uint32_t)(codes >> (2 * (r * CC + c))) & 3u;
+        if (code == 0u) continue;
+        V[r][c] = code == 1u ? 0x7FC00000u : code == 2u ? 0x7F800000u : 0xFF800000u;
+        const int32_t n = code == 1u ? STATE_NAN : STATE_INF;
+        Np[r][c / 2] = (c & 1) ? pack16(lo16(Np[r][c / 2]), n) : pack16(n, hi16(Np[r][c / 2]));
+        dneg0 &= ~(1u << (r * CC + c));
+        to_integer = true;
+      }
+  }
+}
+
+// switch a thread's state from fp32 values (float-assisted path) to (n, X)
+template <int R, int CC>
+__device__ __forceinline__ void values_to_state(uint32_t (&Np)[R][CC / 2], uint32_t (&V)[R][CC]) {
+#pragma unroll
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int p = 0; p < CC / 2; p++) {
+      int32_t n0, n1, x0, x1;
+      bool z;
+      state_from_fp32(V[r][2 * p], n0, x0, z);
+      state_from_fp32(V[r][2 * p + 1], n1, x1, z);
+      V[r][2 * p] = (uint32_t)x0;
+      V[r][2 * p + 1] = (uint32_t)x1;
+      Np[r][p] = pack16(n0, n1);
+    }
+}
+
+// fp32 C values of an R x CC block (row stride ldc), or +0, as raw bits with
+// their packed n; returns whether all of them suit the float-assisted path
+// (finite, and zero or of magnitude >= 2^-FAST_NMAX).
+template <int R, int CC>
+__device__ __forceinline__ bool load_values(const float *C, size_t ldc, bool have_c, uint32_t (&Np)[R][CC / 2],
+                                            uint32_t (&V)[R][CC], uint32_t &dneg0) {
+  dneg0 = 0;
+  bool ok = true;
+#pragma unroll
+  for (int r = 0; r < R; r++) {
+    if (have_c) {
+#pragma unroll
+      for (int q = 0; q < CC / 4; q++) {
+        const uint4 v = reinterpret_cast<const uint4 *>(C + r * ldc)[q];
+        V[r][4 * q] = v.x; V[r][4 * q + 1] = v.y; V[r][4 * q + 2] = v.z; V[r][4 * q + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < CC; c++) V[r][c] = 0u;
+    }
+    int32_t n[CC];
+#pragma unroll
+    for (int c = 0; c < CC; c++) {
+      const uint32_t field = (V[r][c] >> 23) & 0xFFu;
+      const bool zero = (V[r][c] << 1) == 0u;
+      if (zero && V[r][c]) dneg0 |= 1u << (r * CC + c);
+      n[c] = zero ? ZSENT : 127 - (int32_t)field;
+      ok = ok && (zero || (field != 0xFFu && field >= 127u - FAST_NMAX));
+    }
+#pragma unroll
+    for (int p = 0; p < CC / 2; p++) Np[r][p] = pack16(n[2 * p], n[2 * p + 1]);
+  }
+  return ok;
+}
+
 // state of an R x CC block from fp32 C values (row stride ldc), or +0
 template <int R, int CC>
 __device__ __forceinline__ void load_state(const float *C, size_t ldc, bool have_c, uint32_t (&Np)[R][CC / 2],
@@ -503,22 +728,48 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const void
     return sp;
   };
 
+  // accumulator: fp32 bits V on the float-assisted path (FP16 / E4M3 while
+  // the values stay in its range), else the integer state (n, X) in V's place
   uint32_t Np[GR][GCC / 2];
-  int32_t X[GR][GCC];
+  uint32_t V[GR][GCC];
+  int32_t(&X)[GR][GCC] = reinterpret_cast<int32_t(&)[GR][GCC]>(V);
   uint32_t dneg0;
-  load_state<GR, GCC>(C + (size_t)(row0 + rl) * N + col0 + cl, (size_t)N, C != nullptr && out_valid, Np, X, dneg0);
+  bool fast = load_values<GR, GCC>(C + (size_t)(row0 + rl) * N + col0 + cl, (size_t)N, C != nullptr && out_valid, Np,
+                                   V, dneg0);
+  if (!kFloatAssisted<FMT>) fast = false;
+  if (!fast) values_to_state<GR, GCC>(Np, V);
 
   load_chunk(0);
   bool panel_special = __syncthreads_or(store_chunk(panels[0])) != 0;
   for (int j = 0; j < nchunks; j++) {
     if (j + 1 < nchunks) load_chunk(j + 1);
-    mma_chunk<MODEL, FMT, GR, GCC>(panels[j & 1], rl, cl, Np, X, dneg0, panel_special);
+    if constexpr (kFloatAssisted<FMT>) {
+      if (fast) {
+        bool to_integer = false;
+        mma_chunk_fast<MODEL, FMT, GR, GCC>(panels[j & 1], rl, cl, Np, V, dneg0, panel_special, to_integer);
+        if (to_integer) {
+          values_to_state<GR, GCC>(Np, V);
+          fast = false;
+        }
+      } else {
+        mma_chunk<MODEL, FMT, GR, GCC>(panels[j & 1], rl, cl, Np, X, dneg0, panel_special);
+      }
+    } else {
+      mma_chunk<MODEL, FMT, GR, GCC>(panels[j & 1], rl, cl, Np, X, dneg0, panel_special);
+    }
     if (j + 1 < nchunks) panel_special = __syncthreads_or(store_chunk(panels[(j + 1) & 1])) != 0;
   }
 
   // epilogue: store D and the per-16x16-tile xorsum
   uint32_t D[GR][GCC];
-  state_to_fp32<GR, GCC>(Np, X, D);
+  if (fast) {
+#pragma unroll
+    for (int r = 0; r < GR; r++)
+#pragma unroll
+      for (int c = 0; c < GCC; c++) D[r][c] = V[r][c];
+  } else {
+    state_to_fp32<GR, GCC>(Np, X, D);
+  }
   if (out_valid) {
 #pragma unroll
     for (int i = 0; i < GR; i++) {

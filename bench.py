@@ -60,8 +60,14 @@ KERNEL_SOURCES = ("bit_exact_tensor_b200/csrc/mmaemu.cu", "bit_exact_tensor_b200
 HBM_PEAK_GBS = 6557.4  # measured copy bandwidth on this machine's B200s (MEASURED_PEAKS.json)
 DEFAULT_WORKLOAD = "gemm-ampere-fp16-4096"
 PAIRS = (("ampere", "fp16"), ("ampere", "bf16"), ("hopper", "fp16"), ("hopper", "bf16"), ("hopper", "e4m3"))
-WORKLOAD_NAMES = ({DEFAULT_WORKLOAD, "gemm-hopper-bf16-4096", "gemm-hopper-bf16-4096-wide",
-                   "gemm-hopper-e4m3-8192x4096x14336", "tiles-ampere-fp16-4096"}
+E4M3_LAYER = "gemm-hopper-e4m3-8192x4096x14336"
+# variants of the E4M3 layer GEMM: fingerprints only (no D written), verify
+# a claimed D instead of storing it, weights stored [N][K] (B transposed)
+GEMM_MODES = ("fponly", "verify", "wt")
+BATCHED = "gemm-batched-ampere-fp16-8x1024x4096x4096"
+WORKLOAD_NAMES = ({DEFAULT_WORKLOAD, "gemm-hopper-bf16-4096", "gemm-hopper-bf16-4096-wide", E4M3_LAYER,
+                   "tiles-ampere-fp16-4096", BATCHED}
+                  | {f"{E4M3_LAYER}-{m}" for m in GEMM_MODES}
                   | {f"tiles-{m}-{f}-100k" for m, f in PAIRS})
 
 
@@ -73,6 +79,7 @@ def workload_spec(name: str) -> dict:
     def gemm(model, fmt, make, M_, N_, K_, desc):
         eb = 1 if fmt == "e4m3" else 2
         return {"kind": "gemm", "model": model, "fmt": fmt, "make": make, "macs": M_ * N_ * K_, "desc": desc,
+                "mn": (M_, N_), "mode": "store",
                 "h2d": (M_ * K_ + K_ * N_) * eb + M_ * N_ * 4, "d2h": M_ * N_ * 4 + (M_ // 16) * (N_ // 16) * 4,
                 "l2": "inputs larger than L2"}
 
@@ -82,6 +89,28 @@ def workload_spec(name: str) -> dict:
                 "h2d": nt * 256 * (2 * eb + 4), "d2h": nt * 1024,
                 "l2": "inputs larger than L2" if nt * 256 * (2 * eb + 8) > 126e6 else "fits in L2"}
 
+    for mode in GEMM_MODES:
+        if name.endswith("-" + mode):
+            spec = workload_spec(name[: -len(mode) - 1])
+            M_, N_ = spec["mn"]
+            out_d, out_fp = M_ * N_ * 4, (M_ // 16) * (N_ // 16) * 4
+            if mode == "fponly":
+                spec.update(d2h=out_fp, desc=spec["desc"] + ", fingerprints only (D not written)")
+            elif mode == "verify":
+                spec.update(h2d=spec["h2d"] + out_d, d2h=16,
+                            desc=spec["desc"].replace(", fused per-tile xorsum", "")
+                            + ", verify mode (claimed D read and compared, not written)")
+            else:
+                spec.update(desc=spec["desc"] + ", B stored [N][K] (weights layout)")
+            spec["mode"] = mode
+            return spec
+    if name == BATCHED:
+        b_, m_, n_, k_ = 8, 1024, 4096, 4096
+        spec = gemm("ampere", "fp16", lambda r: wl.config_batched(b_, m_, n_, k_, seed=7 + 1000 * r), m_, n_, k_,
+                    f"batched gemm, {b_} independent problems M={m_} N={n_} K={k_} (A, B, C per problem), "
+                    "Ampere FP16 model, N(0,1), fused per-tile xorsum")
+        spec.update(macs=b_ * spec["macs"], h2d=b_ * spec["h2d"], d2h=b_ * spec["d2h"], mode="batched")
+        return spec
     if name == DEFAULT_WORKLOAD:
         return gemm("ampere", "fp16", lambda r: wl.config3(seed=3 + 1000 * r), M, N, K, WORKLOAD)
     if name == "gemm-hopper-bf16-4096":
@@ -90,7 +119,7 @@ def workload_spec(name: str) -> dict:
     if name == "gemm-hopper-bf16-4096-wide":
         return gemm("hopper", "bf16", lambda r: wl.config4(seed=4 + 1000 * r, wide=True), 4096, 4096, 4096,
                     "gemm M=N=K=4096, Hopper BF16 model, log2|x| ~ U[-126, 127], fused per-tile xorsum")
-    if name == "gemm-hopper-e4m3-8192x4096x14336":
+    if name == E4M3_LAYER:
         return gemm("hopper", "e4m3", lambda r: wl.config5(seed=5 + 1000 * r), 8192, 14336, 4096,
                     "gemm M=8192 K=4096 N=14336, Hopper E4M3 model, N(0,1)/sqrt(K), fused per-tile xorsum")
     if name == "tiles-ampere-fp16-4096":
@@ -317,17 +346,39 @@ def run_gpu(args):
         return reduce_max(x, dist, dev)
 
     spec = workload_spec(args.workload)
+    mode = spec.get("mode")
     A_np, B_np, C_np = spec["make"](rank)
-    A = torch.from_numpy(A_np.view(np.uint8 if spec["fmt"] == "e4m3" else np.int16)).to(dev)
-    B = torch.from_numpy(B_np.view(np.uint8 if spec["fmt"] == "e4m3" else np.int16)).to(dev)
+    in_view = np.uint8 if spec["fmt"] == "e4m3" else np.int16
+    if mode == "wt":  # weights layout: B stored as [N][K]
+        B_np = np.ascontiguousarray(B_np.T)
+    A = torch.from_numpy(A_np.view(in_view)).to(dev)
+    B = torch.from_numpy(B_np.view(in_view)).to(dev)
     C = torch.from_numpy(C_np.view(np.int32)).to(dev)
     stream = torch.cuda.current_stream(dev)
+    model, fmt = spec["model"], spec["fmt"]
     if spec["kind"] == "gemm":
         D = torch.empty(C.shape, dtype=torch.float32, device=dev)
-        fp = torch.empty(((C.shape[0] // 16) * (C.shape[1] // 16),), dtype=torch.int32, device=dev)
+        fp = torch.empty(((C.shape[-2] // 16) * (C.shape[-1] // 16),), dtype=torch.int32, device=dev)
+        if mode == "store":
+            def step():
+                mmaemu.gemm(model, fmt, A, B, C, out=D, fp_out=fp)
+        elif mode == "fponly":
+            def step():
+                mmaemu.gemm(model, fmt, A, B, C, fp_out=fp, store_d=False)
+        elif mode == "verify":
+            mmaemu.gemm(model, fmt, A, B, C, out=D, fingerprint=False)  # the claim to verify
+            mism = torch.empty((2,), dtype=torch.int64, device=dev)
 
-        def step():
-            mmaemu.gemm(spec["model"], spec["fmt"], A, B, C, out=D, fp_out=fp)
+            def step():
+                mmaemu.gemm_verify(model, fmt, A, B, C, D, mismatch_out=mism)
+        elif mode == "wt":
+            D3 = D.view(1, *D.shape)
+
+            def step():
+                mmaemu.gemm_batched(model, fmt, A, B.t(), C, out=D3)
+        else:  # batched
+            def step():
+                mmaemu.gemm_batched(model, fmt, A, B, C, out=D)
     else:
         D = torch.empty(C.shape, dtype=torch.float32, device=dev)
 
@@ -366,17 +417,44 @@ def run_gpu(args):
     total_ms = max_over_ranks(total_ms)
     kern_ms = max_over_ranks(sum(per_ms) / len(per_ms))
 
+    if mode == "verify":  # the claim must verify clean
+        count, first = mism.cpu().tolist()
+        if count != 0:
+            raise RuntimeError(f"verify mode found {count} mismatches (first at {first}) in its own result")
+
     # end to end through the public API from pinned host buffers
-    A_h = torch.from_numpy(A_np.view(np.uint8 if spec["fmt"] == "e4m3" else np.int16)).pin_memory()
-    B_h = torch.from_numpy(B_np.view(np.uint8 if spec["fmt"] == "e4m3" else np.int16)).pin_memory()
+    A_h = torch.from_numpy(A_np.view(in_view)).pin_memory()
+    B_h = torch.from_numpy(B_np.view(in_view)).pin_memory()
     C_h = torch.from_numpy(C_np.view(np.int32)).pin_memory()
+    if mode == "verify":
+        Dclaim_h = D.cpu().pin_memory()
+
+    def to_host(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t, non_blocking=True)
+        return h
 
     def e2e_step():
+        if mode == "store":
+            return mmaemu.gemm_host(model, fmt, A_h, B_h, C_h, device=dev)
         if spec["kind"] == "gemm":
-            return mmaemu.gemm_host(spec["model"], spec["fmt"], A_h, B_h, C_h, device=dev)
+            Ad, Bd, Cd = (t.to(dev, non_blocking=True) for t in (A_h, B_h, C_h))
+            if mode == "fponly":
+                out = (None, to_host(mmaemu.gemm(model, fmt, Ad, Bd, Cd, store_d=False)[1]))
+            elif mode == "verify":
+                Dd = Dclaim_h.to(dev, non_blocking=True)
+                out = (to_host(mmaemu.gemm_verify(model, fmt, Ad, Bd, Cd, Dd)[0]), None)
+            elif mode == "wt":
+                Dd, fpd = mmaemu.gemm_batched(model, fmt, Ad, Bd.t(), Cd)
+                out = (to_host(Dd), to_host(fpd))
+            else:
+                Dd, fpd = mmaemu.gemm_batched(model, fmt, Ad, Bd, Cd)
+                out = (to_host(Dd), to_host(fpd))
+            torch.cuda.current_stream(dev).synchronize()
+            return out
         Ad, Bd, Cd = (t.to(dev, non_blocking=True) for t in (A_h, B_h, C_h))
         Dh = torch.empty(C_h.shape, dtype=torch.float32, pin_memory=True)
-        Dh.copy_(mmaemu.tiles(spec["model"], spec["fmt"], Ad, Bd, Cd), non_blocking=True)
+        Dh.copy_(mmaemu.tiles(model, fmt, Ad, Bd, Cd), non_blocking=True)
         torch.cuda.current_stream(dev).synchronize()
         return Dh, None
 

@@ -15,8 +15,8 @@ import ctypes
 import os
 import threading
 
-__all__ = ["MODELS", "FORMATS", "MmaEmuError", "lib", "tiles", "gemm", "xorsum", "xorsum_noalloc", "gemm_host",
-           "set_stream"]
+__all__ = ["MODELS", "FORMATS", "MmaEmuError", "lib", "tiles", "gemm", "gemm_verify", "gemm_batched", "xorsum",
+           "xorsum_noalloc", "gemm_host", "set_stream", "NO_MISMATCH"]
 
 MODELS = {"ampere": 0, "hopper": 1}
 FORMATS = {"fp16": 0, "bf16": 1, "e4m3": 2}
@@ -50,6 +50,12 @@ def lib() -> ctypes.CDLL:
             L.mmaemu_tiles.restype = i32
             L.mmaemu_gemm.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
             L.mmaemu_gemm.restype = i32
+            L.mmaemu_gemm_verify.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+            L.mmaemu_gemm_verify.restype = i32
+            i64 = ctypes.c_longlong
+            L.mmaemu_gemm_strided_batched.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, vp, i64, i64, vp, i64,
+                                                      i64, vp, i64, i64, vp, i64, i64, vp, i64]
+            L.mmaemu_gemm_strided_batched.restype = i32
             L.mmaemu_xorsum.argtypes = [vp, sz, ctypes.POINTER(ctypes.c_uint32)]
             L.mmaemu_xorsum.restype = i32
             L.mmaemu_strerror.argtypes = [i32]
@@ -141,11 +147,7 @@ def tiles(model: str, fmt: str, A, B, C=None, out=None):
     return out
 
 
-def gemm(model: str, fmt: str, A, B, C=None, out=None, fingerprint: bool = True, fp_out=None):
-    """D = C + A B with K walked in ascending 16-wide chunks; returns (D, fp)
-    where fp holds the per-16x16-tile xorsum (None if fingerprint=False)."""
-    torch = _torch()
-    mi, fi = _model_fmt(model, fmt)
+def _gemm_shapes(A, B, C, fmt):
     _check_operand(A, fmt, "A")
     _check_operand(B, fmt, "B")
     if A.dim() != 2 or B.dim() != 2 or A.shape[1] != B.shape[0]:
@@ -156,7 +158,22 @@ def gemm(model: str, fmt: str, A, B, C=None, out=None, fingerprint: bool = True,
         _check_f32(C, "C")
         if tuple(C.shape) != (M, N):
             raise ValueError("C must be [M,N]")
-    if out is None:
+    return M, N, K
+
+
+def gemm(model: str, fmt: str, A, B, C=None, out=None, fingerprint: bool = True, fp_out=None,
+         store_d: bool = True):
+    """D = C + A B with K walked in ascending 16-wide chunks; returns (D, fp)
+    where fp holds the per-16x16-tile xorsum (None if fingerprint=False).
+    store_d=False is the fingerprint-only mode: D is not written (None)."""
+    torch = _torch()
+    mi, fi = _model_fmt(model, fmt)
+    M, N, K = _gemm_shapes(A, B, C, fmt)
+    if not store_d:
+        if not fingerprint:
+            raise ValueError("store_d=False needs fingerprint=True")
+        out = None
+    elif out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=A.device)
     else:
         _check_f32(out, "out")
@@ -166,8 +183,105 @@ def gemm(model: str, fmt: str, A, B, C=None, out=None, fingerprint: bool = True,
                                                            device=A.device)
     set_stream()
     _check(lib().mmaemu_gemm(mi, fi, M, N, K, A.data_ptr(), B.data_ptr(),
-                             C.data_ptr() if C is not None else None, out.data_ptr(),
+                             C.data_ptr() if C is not None else None, out.data_ptr() if out is not None else None,
                              fp.data_ptr() if fp is not None else None), "mmaemu_gemm")
+    return out, fp
+
+
+NO_MISMATCH = -1  # mismatch index word when nothing differs (2^64 - 1 read as int64)
+
+
+def gemm_verify(model: str, fmt: str, A, B, C, D_claimed, fingerprint: bool = False, mismatch_out=None):
+    """Recompute D = C + A B and compare it bit for bit with D_claimed
+    without storing it.  Returns (mismatch, fp): mismatch is an int64 CUDA
+    tensor [count, first] (first = smallest row-major index of a differing
+    element, NO_MISMATCH if none), filled asynchronously; fp the fingerprints
+    of the recomputed D (None if fingerprint=False)."""
+    torch = _torch()
+    mi, fi = _model_fmt(model, fmt)
+    M, N, K = _gemm_shapes(A, B, C, fmt)
+    _check_f32(D_claimed, "D_claimed")
+    if tuple(D_claimed.shape) != (M, N):
+        raise ValueError("D_claimed must be [M,N]")
+    mism = mismatch_out if mismatch_out is not None else torch.empty((2,), dtype=torch.int64, device=A.device)
+    if mism.dtype != torch.int64 or mism.numel() != 2 or not mism.is_cuda:
+        raise TypeError("mismatch_out must be a CUDA int64 tensor of 2 elements")
+    fp = torch.empty(((M // 16) * (N // 16),), dtype=torch.int32, device=A.device) if fingerprint else None
+    set_stream()
+    _check(lib().mmaemu_gemm_verify(mi, fi, M, N, K, A.data_ptr(), B.data_ptr(),
+                                    C.data_ptr() if C is not None else None, D_claimed.data_ptr(),
+                                    fp.data_ptr() if fp is not None else None, mism.data_ptr()),
+           "mmaemu_gemm_verify")
+    return mism, fp
+
+
+def _operand_layout(t, name: str):
+    """(trans, ld, batch stride) of a [batch, rows, cols] (or [rows, cols])
+    view whose rows or columns are contiguous."""
+    rs, cs = t.stride(-2), t.stride(-1)
+    bs = t.stride(0) if t.dim() == 3 else 0
+    if cs == 1 and (rs >= t.shape[-1] or t.shape[-2] == 1):
+        return 0, max(rs, t.shape[-1]), bs
+    if rs == 1 and (cs >= t.shape[-2] or t.shape[-1] == 1):
+        return 1, max(cs, t.shape[-2]), bs
+    raise ValueError(f"{name} needs unit stride along its rows or its columns")
+
+
+def gemm_batched(model: str, fmt: str, A, B, C=None, out=None, fingerprint: bool = True, store_d: bool = True):
+    """Batched D[b] = C[b] + A[b] B[b], each entry with the K-chained
+    arithmetic of gemm.  A: [batch, M, K] or [M, K] (shared), B: [batch, K,
+    N] or [K, N], as strided views: each operand needs unit stride along its
+    rows or along its columns (so A.transpose(-1, -2) views of [K, M] storage
+    work without copies).  C, out: [batch, M, N] with unit column stride.
+    Returns (D, fp) with fp [batch, (M/16)*(N/16)]."""
+    torch = _torch()
+    mi, fi = _model_fmt(model, fmt)
+    for t, name in ((A, "A"), (B, "B")):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if t.dtype not in _in_dtypes()[fmt]:
+            raise TypeError(f"{name} has dtype {t.dtype}, expected one of {_in_dtypes()[fmt]} for {fmt}")
+        if t.dim() not in (2, 3):
+            raise ValueError(f"{name} must be 2-D or 3-D")
+    batch = max(A.shape[0] if A.dim() == 3 else 1, B.shape[0] if B.dim() == 3 else 1)
+    for t, name in ((A, "A"), (B, "B")):
+        if t.dim() == 3 and t.shape[0] != batch:
+            raise ValueError(f"{name} batch size {t.shape[0]} != {batch}")
+    M, K = A.shape[-2:]
+    K2, N = B.shape[-2:]
+    if K != K2:
+        raise ValueError("inner dimensions differ")
+    ta, lda, sa = _operand_layout(A, "A")
+    tb, ldb, sb = _operand_layout(B, "B")
+
+    def f32_layout(t, name):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype not in (torch.float32, torch.int32):
+            raise TypeError(f"{name} must be a CUDA fp32 tensor")
+        if tuple(t.shape[-2:]) != (M, N) or (t.dim() == 3 and t.shape[0] != batch):
+            raise ValueError(f"{name} must be [batch, M, N] or [M, N]")
+        if t.stride(-1) != 1:
+            raise ValueError(f"{name} needs unit column stride")
+        return t.stride(-2), (t.stride(0) if t.dim() == 3 else 0)
+
+    ldc, sc = f32_layout(C, "C") if C is not None else (N, 0)
+    if not store_d:
+        if not fingerprint:
+            raise ValueError("store_d=False needs fingerprint=True")
+        out = None
+    elif out is None:
+        out = torch.empty((batch, M, N), dtype=torch.float32, device=A.device)
+    ldd, sd = f32_layout(out, "out") if out is not None else (N, 0)
+    if out is not None and batch > 1 and sd == 0:
+        raise ValueError("out entries of a batch must not overlap")
+    tiles_per = (M // 16) * (N // 16)
+    fp = torch.empty((batch, tiles_per), dtype=torch.int32, device=A.device) if fingerprint else None
+    set_stream()
+    _check(lib().mmaemu_gemm_strided_batched(
+        mi, fi, ta, tb, M, N, K, batch,
+        A.data_ptr(), lda, sa, B.data_ptr(), ldb, sb,
+        C.data_ptr() if C is not None else None, ldc, sc,
+        out.data_ptr() if out is not None else None, ldd, sd,
+        fp.data_ptr() if fp is not None else None, tiles_per), "mmaemu_gemm_strided_batched")
     return out, fp
 
 

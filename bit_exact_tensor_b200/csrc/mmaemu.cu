@@ -693,12 +693,34 @@ __device__ __forceinline__ uint32_t store_b8(Panel<BM, BN> &P, int n, int h, con
 constexpr int GBM = 64, GBN = 128, GTHREADS = 256, GR = 4, GCC = 8;
 using GPanel = Panel<GBM, GBN>;
 
+// Everything a GEMM launch needs.  Element (m, k) of op(A) sits at
+// A[m * lda + k] (ta == 0) or A[k * lda + m] (ta == 1); element (k, n) of
+// op(B) at B[k * ldb + n] (tb == 0) or B[n * ldb + k] (tb == 1); C, D and
+// Dref are row-major with their own leading dimensions.  Batch b (blockIdx.z)
+// adds b times the batch stride to every pointer.  D, Dref, fp and mism may
+// each be null; C null means +0.
+struct GemmParams {
+  const void *A, *B;
+  const float *C;
+  float *D;
+  const float *Dref;        // claimed result to compare with (verify mode)
+  uint32_t *fp;             // per-16x16-tile xorsum of the computed D
+  unsigned long long *mism; // [0] mismatch count, [1] smallest mismatching index
+  int M, N, K, ta, tb;
+  long long lda, ldb, ldc, ldd, ldr;
+  long long sA, sB, sC, sD, sR, sF;
+};
+
 template <int MODEL, int FMT>
-__global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const void *__restrict__ A, const void *__restrict__ B,
-                                                           const float *__restrict__ C, float *__restrict__ Dout,
-                                                           uint32_t *__restrict__ fp, int M, int N, int K) {
+__global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const GemmParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   GPanel *panels = reinterpret_cast<GPanel *>(smem_raw);
+  constexpr int ESIZE = FMT == FMT_E4M3 ? 1 : 2;
+  const int M = p.M, N = p.N, K = p.K;
+  const size_t bz = blockIdx.z;
+  const void *A = static_cast<const unsigned char *>(p.A) + bz * (size_t)p.sA * ESIZE;
+  const void *B = static_cast<const unsigned char *>(p.B) + bz * (size_t)p.sB * ESIZE;
+  const size_t lda = (size_t)p.lda, ldb = (size_t)p.ldb;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row0 = blockIdx.y * GBM, col0 = blockIdx.x * GBN;
@@ -716,10 +738,14 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const void
 
   const int nchunks = K / 16;
   Raw8<FMT> ra, rb;
+  // 8 k-consecutive elements: one vector load where k is the contiguous
+  // index, else 8 loads that are coalesced across the loader threads
   auto load_chunk = [&](int j) {
-    const int k0 = 16 * j;
-    ra = load_row8<FMT>(A, (size_t)(row0 + am) * K + k0 + 8 * ah, a_valid);
-    rb = load_col8<FMT>(B, (size_t)(k0 + 8 * bh) * N + col0 + bn, (size_t)N, b_valid);
+    const size_t k = 16 * (size_t)j;
+    if (!p.ta) ra = load_row8<FMT>(A, (size_t)(row0 + am) * lda + k + 8 * ah, a_valid);
+    else ra = load_col8<FMT>(A, (k + 8 * ah) * lda + row0 + am, lda, a_valid);
+    if (!p.tb) rb = load_col8<FMT>(B, (k + 8 * bh) * ldb + col0 + bn, ldb, b_valid);
+    else rb = load_row8<FMT>(B, (size_t)(col0 + bn) * ldb + k + 8 * bh, b_valid);
   };
   auto store_chunk = [&](GPanel &P) -> uint32_t {
     uint32_t sp = 0;
@@ -734,8 +760,8 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const void
   uint32_t V[GR][GCC];
   int32_t(&X)[GR][GCC] = reinterpret_cast<int32_t(&)[GR][GCC]>(V);
   uint32_t dneg0;
-  bool fast = load_values<GR, GCC>(C + (size_t)(row0 + rl) * N + col0 + cl, (size_t)N, C != nullptr && out_valid, Np,
-                                   V, dneg0);
+  const float *Cb = p.C ? p.C + bz * (size_t)p.sC + (size_t)(row0 + rl) * p.ldc + col0 + cl : nullptr;
+  bool fast = load_values<GR, GCC>(Cb, (size_t)p.ldc, Cb != nullptr && out_valid, Np, V, dneg0);
   if (!kFloatAssisted<FMT>) fast = false;
   if (!fast) values_to_state<GR, GCC>(Np, V);
 
@@ -760,7 +786,7 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const void
     if (j + 1 < nchunks) panel_special = __syncthreads_or(store_chunk(panels[(j + 1) & 1])) != 0;
   }
 
-  // epilogue: store D and the per-16x16-tile xorsum
+  // epilogue: store D, compare with the claimed D, per-16x16-tile xorsum
   uint32_t D[GR][GCC];
   if (fast) {
 #pragma unroll
@@ -770,15 +796,44 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const void
   } else {
     state_to_fp32<GR, GCC>(Np, X, D);
   }
-  if (out_valid) {
+  if (p.D != nullptr && out_valid) {
+    float *Db = p.D + bz * (size_t)p.sD + (size_t)(row0 + rl) * p.ldd + col0 + cl;
 #pragma unroll
     for (int i = 0; i < GR; i++) {
-      uint4 *dst = reinterpret_cast<uint4 *>(Dout + (size_t)(row0 + rl + i) * N + col0 + cl);
+      uint4 *dst = reinterpret_cast<uint4 *>(Db + (size_t)i * p.ldd);
       dst[0] = make_uint4(D[i][0], D[i][1], D[i][2], D[i][3]);
       dst[1] = make_uint4(D[i][4], D[i][5], D[i][6], D[i][7]);
     }
   }
-  if (fp != nullptr) {
+  if (p.Dref != nullptr) {
+    // bitwise comparison; the smallest mismatching position of the block is
+    // found as the smallest in-block offset (row-major order is preserved)
+    uint32_t count = 0, first = 0xFFFFFFFFu;
+    if (out_valid) {
+      const float *Rb = p.Dref + bz * (size_t)p.sR + (size_t)(row0 + rl) * p.ldr + col0 + cl;
+#pragma unroll
+      for (int i = 0; i < GR; i++) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(Rb + (size_t)i * p.ldr);
+        const uint4 v0 = src[0], v1 = src[1];
+        const uint32_t got[GCC] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int c = GCC - 1; c >= 0; c--)
+          if (got[c] != D[i][c]) {
+            count++;
+            first = min(first, (uint32_t)((rl + i) * GBN + cl + c));
+          }
+      }
+    }
+    count = __reduce_add_sync(0xFFFFFFFFu, count);
+    first = __reduce_min_sync(0xFFFFFFFFu, first);
+    if (lane == 0 && count != 0) {
+      const unsigned long long idx = (unsigned long long)bz * M * N +
+                                     (unsigned long long)(row0 + first / GBN) * N + col0 + first % GBN;
+      atomicAdd(&p.mism[0], (unsigned long long)count);
+      atomicMin(&p.mism[1], idx);
+    }
+  }
+  if (p.fp != nullptr) {
     uint32_t x = 0;
 #pragma unroll
     for (int i = 0; i < GR; i++)
@@ -790,7 +845,7 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const void
     x ^= __shfl_xor_sync(0xFFFFFFFFu, x, 8);
     if (out_valid && (lane & 0xD) == 0) {
       const int tr = (row0 + rl) >> 4, tc = (col0 + cl) >> 4;
-      fp[(size_t)tr * (N >> 4) + tc] = x;
+      p.fp[bz * (size_t)p.sF + (size_t)tr * (N >> 4) + tc] = x;
     }
   }
 }
@@ -894,15 +949,80 @@ bool valid_pair(int model, int fmt) {
   return !(model == MMAEMU_AMPERE && fmt == MMAEMU_E4M3);
 }
 
+#define MMAEMU_DISPATCH(model, fmt, CALL)                                               \
+  do {                                                                                  \
+    if (model == MMAEMU_AMPERE && fmt == MMAEMU_FP16) return CALL(0, 0);                \
+    if (model == MMAEMU_AMPERE && fmt == MMAEMU_BF16) return CALL(0, 1);                \
+    if (model == MMAEMU_HOPPER && fmt == MMAEMU_FP16) return CALL(1, 0);                \
+    if (model == MMAEMU_HOPPER && fmt == MMAEMU_BF16) return CALL(1, 1);                \
+    if (model == MMAEMU_HOPPER && fmt == MMAEMU_E4M3) return CALL(1, 2);                \
+    return MMAEMU_EINVAL;                                                               \
+  } while (0)
+
 template <int MODEL, int FMT>
-int launch_gemm(int M, int N, int K, const void *A, const void *B, const float *C, float *D, uint32_t *fp) {
+int launch_gemm(const mmaemu::GemmParams &p, int batch) {
   const size_t smem = 2 * sizeof(mmaemu::GPanel);
   auto kern = mmaemu::gemm_kernel<MODEL, FMT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return MMAEMU_ECUDA;
-  dim3 grid((N + mmaemu::GBN - 1) / mmaemu::GBN, (M + mmaemu::GBM - 1) / mmaemu::GBM);
-  kern<<<grid, mmaemu::GTHREADS, smem, t_stream>>>(A, B, C, D, fp, M, N, K);
+  dim3 grid((p.N + mmaemu::GBN - 1) / mmaemu::GBN, (p.M + mmaemu::GBM - 1) / mmaemu::GBM, batch);
+  kern<<<grid, mmaemu::GTHREADS, smem, t_stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
+}
+
+// Shape, layout and alignment rules shared by the GEMM entry points.
+int validate_gemm(const mmaemu::GemmParams &p, long long batch) {
+  if (p.M <= 0 || p.N <= 0 || p.K <= 0 || (p.M & 15) || (p.N & 15) || (p.K & 15)) return MMAEMU_EINVAL;
+  if (batch < 1 || batch > 65535) return MMAEMU_EINVAL;
+  if ((long long)p.M / mmaemu::GBM >= 65535) return MMAEMU_EINVAL;
+  if (!p.A || !p.B) return MMAEMU_EINVAL;
+  if (!p.D && !p.fp && !p.Dref) return MMAEMU_EINVAL;  // nothing to produce
+  if (p.Dref && !p.mism) return MMAEMU_EINVAL;
+  if ((p.ta != 0 && p.ta != 1) || (p.tb != 0 && p.tb != 1)) return MMAEMU_EINVAL;
+  // leading dimensions cover a row of the stored matrix; vector-loaded rows
+  // (A not transposed, B transposed, C, D, Dref) start on 16-byte boundaries
+  const long long a_row = p.ta ? p.M : p.K, b_row = p.tb ? p.K : p.N;
+  if (p.lda < a_row || p.ldb < b_row) return MMAEMU_EINVAL;
+  constexpr long long vec = 8;  // elements per operand vector load (16 B of fp16/bf16, 8 B of e4m3)
+  if (!aligned16(p.A) || !aligned16(p.B)) return MMAEMU_EINVAL;
+  if (!p.ta && (p.lda % vec || p.sA % vec)) return MMAEMU_EINVAL;
+  if (p.tb && (p.ldb % vec || p.sB % vec)) return MMAEMU_EINVAL;
+  if (p.sA < 0 || p.sB < 0 || p.sC < 0 || p.sD < 0 || p.sR < 0 || p.sF < 0) return MMAEMU_EINVAL;
+  struct F32 { const void *ptr; long long ld, stride; };
+  const F32 mats[3] = {{p.C, p.ldc, p.sC}, {p.D, p.ldd, p.sD}, {p.Dref, p.ldr, p.sR}};
+  for (const F32 &m : mats) {
+    if (!m.ptr) continue;
+    if (!aligned16(m.ptr) || m.ld < p.N || m.ld % 4 || m.stride % 4) return MMAEMU_EINVAL;
+  }
+  if (p.fp && ((uintptr_t)p.fp & 3u)) return MMAEMU_EINVAL;
+  if (batch > 1 && p.fp && p.sF < (long long)(p.M / 16) * (p.N / 16)) return MMAEMU_EINVAL;
+  return MMAEMU_OK;
+}
+
+int run_gemm(int model, int fmt, mmaemu::GemmParams &p, long long batch) {
+  if (!valid_pair(model, fmt)) return MMAEMU_EINVAL;
+  int rc = validate_gemm(p, batch);
+  if (rc != MMAEMU_OK) return rc;
+  rc = check_device();
+  if (rc != MMAEMU_OK) return rc;
+  if (p.Dref) {
+    // count 0, smallest index all-ones ("none")
+    if (cudaMemsetAsync(p.mism, 0, sizeof(unsigned long long), t_stream) != cudaSuccess ||
+        cudaMemsetAsync(p.mism + 1, 0xFF, sizeof(unsigned long long), t_stream) != cudaSuccess)
+      return MMAEMU_ECUDA;
+  }
+#define CALL_GEMM(M_, F_) launch_gemm<M_, F_>(p, (int)batch)
+  MMAEMU_DISPATCH(model, fmt, CALL_GEMM);
+#undef CALL_GEMM
+}
+
+mmaemu::GemmParams row_major_params(int M, int N, int K, const void *A, const void *B, const float *C, float *D,
+                                    uint32_t *fp) {
+  mmaemu::GemmParams p{};
+  p.A = A; p.B = B; p.C = C; p.D = D; p.fp = fp;
+  p.M = M; p.N = N; p.K = K;
+  p.lda = K; p.ldb = N; p.ldc = N; p.ldd = N; p.ldr = N;
+  return p;
 }
 
 template <int MODEL, int FMT>
@@ -922,15 +1042,6 @@ int launch_tiles(const void *A, const void *B, const float *C, float *D, size_t 
   return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
 }
 
-#define MMAEMU_DISPATCH(model, fmt, CALL)                                               \
-  do {                                                                                  \
-    if (model == MMAEMU_AMPERE && fmt == MMAEMU_FP16) return CALL(0, 0);                \
-    if (model == MMAEMU_AMPERE && fmt == MMAEMU_BF16) return CALL(0, 1);                \
-    if (model == MMAEMU_HOPPER && fmt == MMAEMU_FP16) return CALL(1, 0);                \
-    if (model == MMAEMU_HOPPER && fmt == MMAEMU_BF16) return CALL(1, 1);                \
-    if (model == MMAEMU_HOPPER && fmt == MMAEMU_E4M3) return CALL(1, 2);                \
-    return MMAEMU_EINVAL;                                                               \
-  } while (0)
 
 }  // namespace
 
@@ -957,20 +1068,33 @@ int mmaemu_tiles(int model, int fmt, const void *A, const void *B, const float *
 
 int mmaemu_gemm(int model, int fmt, int M, int N, int K, const void *A, const void *B, const float *C, float *D,
                 uint32_t *fingerprint_out) {
-  if (!valid_pair(model, fmt)) return MMAEMU_EINVAL;
-  if (M <= 0 || N <= 0 || K <= 0 || (M & 15) || (N & 15) || (K & 15)) return MMAEMU_EINVAL;
-  if ((int64_t)M * K >= ((int64_t)1 << 31) || (int64_t)K * N >= ((int64_t)1 << 31) ||
-      (int64_t)M * N >= ((int64_t)1 << 31))
-    return MMAEMU_EINVAL;
-  if (!A || !B || !D) return MMAEMU_EINVAL;
-  if (!aligned16(A) || !aligned16(B) || !aligned16(D) || (C && !aligned16(C)) ||
-      (fingerprint_out && !aligned16(fingerprint_out)))
-    return MMAEMU_EINVAL;
-  const int rc = check_device();
-  if (rc != MMAEMU_OK) return rc;
-#define CALL_GEMM(M_, F_) launch_gemm<M_, F_>(M, N, K, A, B, C, D, fingerprint_out)
-  MMAEMU_DISPATCH(model, fmt, CALL_GEMM);
-#undef CALL_GEMM
+  mmaemu::GemmParams p = row_major_params(M, N, K, A, B, C, D, fingerprint_out);
+  if (!D && !fingerprint_out) return MMAEMU_EINVAL;
+  return run_gemm(model, fmt, p, 1);
+}
+
+int mmaemu_gemm_verify(int model, int fmt, int M, int N, int K, const void *A, const void *B, const float *C,
+                       const float *D_claimed, uint32_t *fingerprint_out, unsigned long long *mismatch_out) {
+  if (!D_claimed || !mismatch_out) return MMAEMU_EINVAL;
+  mmaemu::GemmParams p = row_major_params(M, N, K, A, B, C, nullptr, fingerprint_out);
+  p.Dref = D_claimed;
+  p.mism = mismatch_out;
+  return run_gemm(model, fmt, p, 1);
+}
+
+int mmaemu_gemm_strided_batched(int model, int fmt, int trans_a, int trans_b, int M, int N, int K, int batch,
+                                const void *A, long long lda, long long stride_a, const void *B, long long ldb,
+                                long long stride_b, const float *C, long long ldc, long long stride_c, float *D,
+                                long long ldd, long long stride_d, uint32_t *fingerprint_out,
+                                long long stride_fp) {
+  mmaemu::GemmParams p{};
+  p.A = A; p.B = B; p.C = C; p.D = D; p.fp = fingerprint_out;
+  p.M = M; p.N = N; p.K = K; p.ta = trans_a; p.tb = trans_b;
+  p.lda = lda; p.ldb = ldb; p.ldc = C ? ldc : N; p.ldd = D ? ldd : N; p.ldr = N;
+  p.sA = stride_a; p.sB = stride_b; p.sC = C ? stride_c : 0; p.sD = D ? stride_d : 0;
+  p.sF = fingerprint_out ? stride_fp : 0;
+  if (!D && !fingerprint_out) return MMAEMU_EINVAL;
+  return run_gemm(model, fmt, p, batch);
 }
 
 int mmaemu_xorsum(const void *D, size_t n, uint32_t *out_host) {

@@ -251,6 +251,17 @@ def config5(seed: int = 5, M: int = 8192, N: int = 14336, K: int = 4096):
     return gemm_normal(M, N, K, "e4m3", seed, scale=1.0 / np.sqrt(K))
 
 
+def config_batched(batch: int, M: int, N: int, K: int, seed: int = 7, fmt: str = "fp16"):
+    """A batch of independent GEMMs (per-expert or per-head MatMuls of a
+    model layer): A [batch,M,K], B [batch,K,N] ~ N(0,1), C [batch,M,N] ~
+    N(0,1) in fp32."""
+    rng = np.random.default_rng(seed)
+    A = to_bits(rng.standard_normal((batch, M, K), dtype=np.float32), fmt)
+    B = to_bits(rng.standard_normal((batch, K, N), dtype=np.float32), fmt)
+    C = f32_bits(rng.standard_normal((batch, M, N), dtype=np.float32))
+    return A, B, C
+
+
 # ---------------------------------------------------------------------------
 # special values (parity only)
 # ---------------------------------------------------------------------------

@@ -14,9 +14,11 @@
  * Common rules for every call below:
  *  - All data pointers are DEVICE pointers owned by the caller; the library
  *    never frees, keeps or writes outside them.  Inputs are never modified.
- *  - Matrices are dense and row-major.  fp16 and bf16 elements are 2 bytes,
- *    e4m3 elements 1 byte (OCP FP8 E4M3: no infinities, S.1111.111 is NaN),
- *    C and D are IEEE fp32.  Every pointer must be 16-byte aligned.
+ *  - Matrices are dense and row-major (mmaemu_gemm_strided_batched also
+ *    takes transposed and strided layouts).  fp16 and bf16 elements are 2
+ *    bytes, e4m3 elements 1 byte (OCP FP8 E4M3: no infinities, S.1111.111 is
+ *    NaN), C and D are IEEE fp32.  Every pointer must be 16-byte aligned,
+ *    except where a call states otherwise.
  *  - Work is enqueued on the stream set with mmaemu_set_stream for the
  *    calling host thread (default: the legacy default stream) and is
  *    asynchronous unless stated otherwise.  Errors of the kernels themselves
@@ -80,15 +82,66 @@ int mmaemu_tiles(int model, int fmt, const void *A, const void *B, const float *
  *   d_0 = C[m][n];  d_{j+1} = MMA16(A[m][16j..16j+15], B[16j..16j+15][n], d_j).
  *   A: [M][K] in fmt; B: [K][N] in fmt; C, D: [M][N] fp32; C may be NULL (+0)
  *   and may equal D (in place); no other overlap.
- *   M, N, K: positive multiples of 16, M*K, K*N and M*N below 2^31.
+ *   M, N, K: positive multiples of 16; M / 64 below 65535.
  *   fingerprint_out: NULL, or [(M/16)*(N/16)] uint32 written with the
  *   xorsum (XOR of the 256 fp32 bit patterns) of each 16x16 tile of D, tiles
  *   in row-major tile-grid order -- the AEGIS xorsum fingerprint, fused into
  *   the epilogue.
- * Errors: MMAEMU_EINVAL, MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED; on error nothing
- * is enqueued.                                                              */
+ *   D may be NULL when fingerprint_out is not: the fingerprints are computed
+ *   and nothing of D is written (fingerprint-only mode).
+ * Errors: MMAEMU_EINVAL (also for D and fingerprint_out both NULL),
+ * MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED; on error nothing is enqueued.          */
 int mmaemu_gemm(int model, int fmt, int M, int N, int K, const void *A, const void *B,
                 const float *C, float *D, uint32_t *fingerprint_out);
+
+/* Verify mode of mmaemu_gemm: recomputes D = C + A . B exactly as
+ * mmaemu_gemm does and compares it, bit for bit, with a claimed result
+ * instead of storing it -- the auditor's side of the workflow in the Hawkeye
+ * notes ("relation to the verifiable-ML workflow": the simulator as oracle,
+ * compared with the MatMul outputs a provider publishes), where any
+ * difference means the claimed computation was not the modelled one.
+ *   D_claimed: [M][N] fp32, row-major, 16-byte aligned; only read.  Every bit
+ *   counts: a NaN with another payload, or -0 for +0, is a mismatch.
+ *   mismatch_out: device array of 2 unsigned 64-bit words, overwritten (it
+ *   needs no initialisation): [0] = number of mismatching elements, [1] =
+ *   smallest row-major index m*N + n among them, or 2^64 - 1 if none.
+ *   fingerprint_out: NULL, or the fingerprints of the RECOMPUTED D, as in
+ *   mmaemu_gemm.
+ * Other arguments and rules as mmaemu_gemm.  Asynchronous: read mismatch_out
+ * after the stream has reached this call.  Errors: MMAEMU_EINVAL (also NULL
+ * D_claimed or mismatch_out), MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED.           */
+int mmaemu_gemm_verify(int model, int fmt, int M, int N, int K, const void *A, const void *B,
+                       const float *C, const float *D_claimed, uint32_t *fingerprint_out,
+                       unsigned long long *mismatch_out);
+
+/* mmaemu_gemm over other storage layouts and batches of independent
+ * problems, each with the same K-chained arithmetic -- for MatMuls as they
+ * appear in model layers (the Hawkeye notes' "design trade-offs": real
+ * training shapes, batches and layouts have to be mapped onto the 16x16
+ * MMA tiles).  For batch entry b (0 <= b < batch), with every stride and
+ * leading dimension counted in ELEMENTS:
+ *   op(A)[m][k] = A[b*stride_a + m*lda + k]   if trans_a == 0  (lda >= K)
+ *               = A[b*stride_a + k*lda + m]   if trans_a == 1  (lda >= M)
+ *   op(B)[k][n] = B[b*stride_b + k*ldb + n]   if trans_b == 0  (ldb >= N)
+ *               = B[b*stride_b + n*ldb + k]   if trans_b == 1  (ldb >= K)
+ *   C[b*stride_c + m*ldc + n] (C may be NULL: +0), D[b*stride_d + m*ldd + n]
+ *   fingerprint_out[b*stride_fp + (m/16)*(N/16) + n/16] (may be NULL;
+ *   stride_fp >= (M/16)*(N/16) when batch > 1)
+ * D may be NULL when fingerprint_out is not (fingerprint-only).  Strides may
+ * be 0 for inputs shared by every batch entry (e.g. one B for all); the D
+ * and fingerprint regions of different entries must not overlap.
+ * Layout rules (MMAEMU_EINVAL otherwise): A and B 16-byte aligned; when A is
+ * not transposed lda and stride_a are multiples of 8, and likewise ldb and
+ * stride_b when B is transposed (those rows are read as 8-element vectors);
+ * C and D 16-byte aligned with ldc, ldd >= N and ldc, ldd, stride_c,
+ * stride_d multiples of 4; fingerprint_out 4-byte aligned; strides >= 0;
+ * 1 <= batch <= 65535; trans_a, trans_b in {0, 1}; M, N, K as mmaemu_gemm.
+ * Errors: MMAEMU_EINVAL, MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED.                 */
+int mmaemu_gemm_strided_batched(int model, int fmt, int trans_a, int trans_b, int M, int N, int K,
+                                int batch, const void *A, long long lda, long long stride_a,
+                                const void *B, long long ldb, long long stride_b, const float *C,
+                                long long ldc, long long stride_c, float *D, long long ldd,
+                                long long stride_d, uint32_t *fingerprint_out, long long stride_fp);
 
 /* xorsum of n 32-bit words at device pointer D (the AEGIS fingerprint of a
  * whole tensor), written to *out_host.  SYNCHRONOUS: returns after the

@@ -40,8 +40,9 @@ def L():
 
 
 def test_header_declares_the_boundary():
-    assert declared_functions() == ["mmaemu_gemm", "mmaemu_set_stream", "mmaemu_strerror", "mmaemu_tiles",
-                                    "mmaemu_xorsum", "mmaemu_xorsum_noalloc"]
+    assert declared_functions() == ["mmaemu_gemm", "mmaemu_gemm_strided_batched", "mmaemu_gemm_verify",
+                                    "mmaemu_set_stream", "mmaemu_strerror", "mmaemu_tiles", "mmaemu_xorsum",
+                                    "mmaemu_xorsum_noalloc"]
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -80,7 +81,38 @@ def test_invalid_arguments_rejected_before_any_device_work(L):
     assert L.mmaemu_gemm(1, 0, 16, 16, -16, p, p, None, p, None) == EINVAL
     assert L.mmaemu_gemm(1, 0, 16, 16, 16, None, p, None, p, None) == EINVAL
     assert L.mmaemu_gemm(1, 0, 16, 16, 16, p + 2, p, None, p, None) == EINVAL
-    assert L.mmaemu_gemm(1, 0, 1 << 16, 1 << 16, 16, p, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(1, 0, 65535 * 64, 16, 16, p, p, None, p, None) == EINVAL  # grid rows
+    assert L.mmaemu_gemm(1, 0, 16, 16, 16, p, p, None, None, None) == EINVAL  # nothing to produce
+    # verify mode: the claimed D and the mismatch words are required
+    assert L.mmaemu_gemm_verify(1, 0, 16, 16, 16, p, p, None, None, None, p) == EINVAL
+    assert L.mmaemu_gemm_verify(1, 0, 16, 16, 16, p, p, None, p, None, None) == EINVAL
+    assert L.mmaemu_gemm_verify(0, 2, 16, 16, 16, p, p, None, p, None, p) == EINVAL
+    assert L.mmaemu_gemm_verify(1, 0, 16, 16, 16, p, p, None, p + 8, None, p) == EINVAL
+
+    def sb(ta=0, tb=0, M=16, N=16, K=16, batch=1, lda=16, sa=0, ldb=16, sbb=0, C=None, ldc=16, sc=0, D=p, ldd=16,
+           sd=0, fp=None, sf=0, A=p):
+        f = L.mmaemu_gemm_strided_batched
+        f.argtypes = [ctypes.c_int] * 8 + [ctypes.c_void_p, ctypes.c_longlong, ctypes.c_longlong] * 4 + [
+            ctypes.c_void_p, ctypes.c_longlong]
+        return f(1, 0, ta, tb, M, N, K, batch, A, lda, sa, p, ldb, sbb, C, ldc, sc, D, ldd, sd, fp, sf)
+
+    assert sb(ta=2) == EINVAL
+    assert sb(tb=-1) == EINVAL
+    assert sb(lda=8) == EINVAL                 # lda < K
+    assert sb(ta=1, lda=8) == EINVAL           # lda < M
+    assert sb(lda=20) == EINVAL                # vector-loaded rows need lda % 8 == 0
+    assert sb(sa=4, batch=2, sd=256) == EINVAL  # ... and stride_a % 8 == 0
+    assert sb(tb=1, ldb=24 + 4) == EINVAL      # transposed B rows are vector-loaded too
+    assert sb(ldd=18) == EINVAL                # ldd % 4
+    assert sb(ldd=8) == EINVAL                 # ldd < N
+    assert sb(C=p, ldc=16, sc=2, batch=2, sd=256) == EINVAL
+    assert sb(batch=0) == EINVAL
+    assert sb(batch=65536, sd=256) == EINVAL
+    assert sb(sa=-8) == EINVAL
+    assert sb(D=None, fp=None) == EINVAL
+    assert sb(D=None, fp=p + 2) == EINVAL      # fingerprints are 4-byte aligned
+    assert sb(D=None, fp=p, batch=2, sf=0) == EINVAL  # fingerprint regions overlap
+    assert sb(A=p + 8) == EINVAL
     assert L.mmaemu_tiles(0, 2, p, p, None, p, 1) == EINVAL
     assert L.mmaemu_tiles(0, 0, p, p, None, None, 1) == EINVAL
     assert L.mmaemu_tiles(0, 0, p, p, p + 4, p, 1) == EINVAL

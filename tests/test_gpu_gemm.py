@@ -77,6 +77,9 @@ def accumulator_edge_inputs(fmt, seed):
                    unchanged through three chunks before products arrive;
       rows 32-63   products cancelling in pairs (A[:, 2j+1] = -A[:, 2j],
                    B[2j+1] = B[2j]), so every group sum is C's part alone;
+                   rows 40-47 also have C = +-0 and zeros in the second
+                   half of every chunk (an Ampere stage-1 sum of zero
+                   followed by a stage of zero products);
       rows 64-95   A zero in every chunk;
       rows 96-111  subnormal A (against subnormal B in columns 16-31, the
                    smallest products there are);
@@ -95,6 +98,8 @@ def accumulator_edge_inputs(fmt, seed):
     A[0:32, 0:48] = zeros((32, 48))
     A[32:64, 1::2] = A[32:64, 0::2] ^ A.dtype.type(sign)
     B[1::2, :] = B[0::2, :]
+    for j in range(K // 16):  # rows 40-47: the second half of every chunk zero
+        A[40:48, 16 * j + 8:16 * j + 16] = 0
     A[64:80, :] = sign
     A[80:96, :] = zeros((16, K))
     A[96:112, :] = wl.random_subnormals(rng, (16, K), fmt)
@@ -110,6 +115,7 @@ def accumulator_edge_inputs(fmt, seed):
     pick = rng.random((M, N)) < 0.7
     C[pick] = pool[rng.integers(0, pool.size, size=int(pick.sum()))]
     C[64:80, 0:16] = np.where(rng.random((16, 16)) < 0.5, 0x80000000, 0).astype(np.uint32)
+    C[40:48, :] = np.where(rng.random((8, N)) < 0.5, 0x80000000, 0).astype(np.uint32)
     return A, B, C
 
 

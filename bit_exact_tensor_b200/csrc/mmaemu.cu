@@ -508,26 +508,16 @@ __device__ __forceinline__ void values_to_state(uint32_t (&Np)[R][CC / 2], uint3
     }
 }
 
-// fp32 C values of an R x CC block (row stride ldc), or +0, as raw bits with
-// their packed n; returns whether all of them suit the float-assisted path
-// (zero, or of magnitude in [2^-FAST_NMAX, 2^FAST_EMAX)).
+// Packed n and -0 mask of an R x CC block of fp32 values V (raw bits); returns
+// whether all of them suit the float-assisted path (zero, or of magnitude in
+// [2^-FAST_NMAX, 2^FAST_EMAX)).
 template <int R, int CC>
-__device__ __forceinline__ bool load_values(const float *C, size_t ldc, bool have_c, uint32_t (&Np)[R][CC / 2],
-                                            uint32_t (&V)[R][CC], uint32_t &dneg0) {
+__device__ __forceinline__ bool classify_values(const uint32_t (&V)[R][CC], uint32_t (&Np)[R][CC / 2],
+                                                uint32_t &dneg0) {
   dneg0 = 0;
   bool ok = true;
 #pragma unroll
   for (int r = 0; r < R; r++) {
-    if (have_c) {
-#pragma unroll
-      for (int q = 0; q < CC / 4; q++) {
-        const uint4 v = reinterpret_cast<const uint4 *>(C + r * ldc)[q];
-        V[r][4 * q] = v.x; V[r][4 * q + 1] = v.y; V[r][4 * q + 2] = v.z; V[r][4 * q + 3] = v.w;
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < CC; c++) V[r][c] = 0u;
-    }
     int32_t n[CC];
 #pragma unroll
     for (int c = 0; c < CC; c++) {
@@ -541,6 +531,32 @@ __device__ __forceinline__ bool load_values(const float *C, size_t ldc, bool hav
     for (int p = 0; p < CC / 2; p++) Np[r][p] = pack16(n[2 * p], n[2 * p + 1]);
   }
   return ok;
+}
+
+// raw fp32 bits of an R x CC block (row stride ldc), or +0 if !have_c
+template <int R, int CC>
+__device__ __forceinline__ void load_bits(const float *C, size_t ldc, bool have_c, uint32_t (&V)[R][CC]) {
+#pragma unroll
+  for (int r = 0; r < R; r++) {
+    if (have_c) {
+#pragma unroll
+      for (int q = 0; q < CC / 4; q++) {
+        const uint4 v = reinterpret_cast<const uint4 *>(C + r * ldc)[q];
+        V[r][4 * q] = v.x; V[r][4 * q + 1] = v.y; V[r][4 * q + 2] = v.z; V[r][4 * q + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < CC; c++) V[r][c] = 0u;
+    }
+  }
+}
+
+// fp32 C values of an R x CC block as raw bits with their packed n
+template <int R, int CC>
+__device__ __forceinline__ bool load_values(const float *C, size_t ldc, bool have_c, uint32_t (&Np)[R][CC / 2],
+                                            uint32_t (&V)[R][CC], uint32_t &dneg0) {
+  load_bits<R, CC>(C, ldc, have_c, V);
+  return classify_values<R, CC>(V, Np, dneg0);
 }
 
 // state of an R x CC block from fp32 C values (row stride ldc), or +0
@@ -839,7 +855,7 @@ constexpr int TWARPS = 8, TR = 2, TCC = 4;
 using TPanel = Panel<16, 16>;
 
 template <int MODEL, int FMT>
-__global__ void __launch_bounds__(TWARPS * 32) tiles_kernel(const void *__restrict__ A, const void *__restrict__ B,
+__global__ void __launch_bounds__(TWARPS * 32, 3) tiles_kernel(const void *__restrict__ A, const void *__restrict__ B,
                                                             const float *__restrict__ C, float *__restrict__ Dout,
                                                             size_t ntiles) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -847,24 +863,68 @@ __global__ void __launch_bounds__(TWARPS * 32) tiles_kernel(const void *__restri
   TPanel &P = reinterpret_cast<TPanel *>(smem_raw)[warp];
   const int rl = (lane >> 2) * TR, cl = (lane & 3) * TCC;
   const int lm = lane & 15, lh = lane >> 4;
-  for (size_t t = (size_t)blockIdx.x * TWARPS + warp; t < ntiles; t += (size_t)gridDim.x * TWARPS) {
-    const Raw8<FMT> ra = load_row8<FMT>(A, t * 256 + lm * 16 + 8 * lh, true);
-    const Raw8<FMT> rb = load_col8<FMT>(B, t * 256 + (8 * lh) * 16 + lm, 16, true);
-    uint32_t Np[TR][TCC / 2];
-    int32_t X[TR][TCC];
-    uint32_t dneg0;
-    load_state<TR, TCC>(C + t * 256 + rl * 16 + cl, 16, C != nullptr, Np, X, dneg0);
+  const size_t stride = (size_t)gridDim.x * TWARPS;
+  size_t t = (size_t)blockIdx.x * TWARPS + warp;
+  if (t >= ntiles) return;  // warp-uniform
+
+  // raw operands and C of the next tile are loaded while this one computes
+  auto load_a = [&](size_t u) { return load_row8<FMT>(A, u * 256 + lm * 16 + 8 * lh, true); };
+  auto load_b = [&](size_t u) { return load_col8<FMT>(B, u * 256 + (8 * lh) * 16 + lm, 16, true); };
+  auto load_c = [&](size_t u, uint32_t(&cv)[TR][TCC]) {
+    load_bits<TR, TCC>(C + u * 256 + rl * 16 + cl, 16, C != nullptr, cv);
+  };
+  Raw8<FMT> ra = load_a(t), rb = load_b(t);
+  uint32_t cnext[TR][TCC];
+  load_c(t, cnext);
+  uint32_t Np[TR][TCC / 2];
+  uint32_t V[TR][TCC];
+  int32_t(&X)[TR][TCC] = reinterpret_cast<int32_t(&)[TR][TCC]>(V);
+  uint32_t dneg0;
+  for (;;) {
+#pragma unroll
+    for (int i = 0; i < TR; i++)
+#pragma unroll
+      for (int c = 0; c < TCC; c++) V[i][c] = cnext[i][c];
+    bool fast = classify_values<TR, TCC>(V, Np, dneg0);
+    if (!kFloatAssisted<FMT>) fast = false;
+    if (!fast) values_to_state<TR, TCC>(Np, V);
     __syncwarp();  // the previous tile's reads of P are done
     uint32_t sp = store_a8<MODEL, FMT>(P, lm, lh, ra);
     sp |= store_b8<FMT>(P, lm, lh, rb);
     const bool panel_special = __any_sync(0xFFFFFFFFu, sp != 0);
     __syncwarp();
-    mma_chunk<MODEL, FMT, TR, TCC>(P, rl, cl, Np, X, dneg0, panel_special);
+    const size_t next = t + stride;
+    if (next < ntiles) {
+      ra = load_a(next);
+      rb = load_b(next);
+      load_c(next, cnext);
+    }
     uint32_t D[TR][TCC];
-    state_to_fp32<TR, TCC>(Np, X, D);
+    if constexpr (kFloatAssisted<FMT>) {
+      bool to_integer = false;
+      if (fast) {
+        mma_chunk_fast<MODEL, FMT, TR, TCC>(P, rl, cl, Np, V, dneg0, panel_special, to_integer);
+        if (to_integer) values_to_state<TR, TCC>(Np, V);
+      } else {
+        mma_chunk<MODEL, FMT, TR, TCC>(P, rl, cl, Np, X, dneg0, panel_special);
+      }
+      if (fast && !to_integer) {
+#pragma unroll
+        for (int i = 0; i < TR; i++)
+#pragma unroll
+          for (int c = 0; c < TCC; c++) D[i][c] = V[i][c];
+      } else {
+        state_to_fp32<TR, TCC>(Np, X, D);
+      }
+    } else {
+      mma_chunk<MODEL, FMT, TR, TCC>(P, rl, cl, Np, X, dneg0, panel_special);
+      state_to_fp32<TR, TCC>(Np, X, D);
+    }
 #pragma unroll
     for (int i = 0; i < TR; i++)
       *reinterpret_cast<uint4 *>(Dout + t * 256 + (rl + i) * 16 + cl) = make_uint4(D[i][0], D[i][1], D[i][2], D[i][3]);
+    t = next;
+    if (t >= ntiles) break;
   }
 }
 

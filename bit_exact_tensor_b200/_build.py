@@ -8,7 +8,9 @@ import subprocess
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "mmaemu.cu")
-DEPS = [SRC, os.path.join(PKG, "csrc", "mmaemu_core.cuh"), os.path.join(ROOT, "include", "mmaemu.h")]
+SOURCES = [SRC, os.path.join(PKG, "csrc", "probe.cpp")]
+DEPS = SOURCES + [os.path.join(PKG, "csrc", "mmaemu_core.cuh"), os.path.join(ROOT, "include", "mmaemu.h"),
+                  os.path.join(ROOT, "include", "mmaemu_probe.h")]
 LIB = os.path.join(PKG, "libmmaemu.so")
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
@@ -33,7 +35,7 @@ def build_library(force: bool = False, verbose: bool = False) -> str:
     if not force and not needs_build():
         return LIB
     tmp = LIB + f".{os.getpid()}.tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), SRC, "-o", tmp]
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), *SOURCES, "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)

@@ -951,6 +951,93 @@ __global__ void __launch_bounds__(256) xorsum_kernel(const uint4 *__restrict__ v
   }
 }
 
+// ---------------------------------------------------------------------------
+// B200's own tensor-core MMA on the same tile batches (a probe target, not
+// part of the emulation): one warp per 16x16x16 tile, two mma.sync
+// m16n8k16 (FP16/BF16) or m16n8k32 with k >= 16 zero (E4M3) per tile, fp32
+// accumulate.  Fragment layouts are those of the PTX mma.sync description.
+// ---------------------------------------------------------------------------
+template <int FMT>
+__global__ void __launch_bounds__(256) native_tiles_kernel(const void *__restrict__ A, const void *__restrict__ B,
+                                                         const float *__restrict__ C, float *__restrict__ D,
+                                                         size_t ntiles) {
+  const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+  for (size_t t = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < ntiles;
+       t += (size_t)gridDim.x * (blockDim.x >> 5)) {
+    uint32_t a[4], b[2][2];
+    if constexpr (FMT == FMT_E4M3) {
+      const uint8_t *At = static_cast<const uint8_t *>(A) + t * 256;
+      const uint8_t *Bt = static_cast<const uint8_t *>(B) + t * 256;
+      auto row4 = [&](int m) { return *reinterpret_cast<const uint32_t *>(At + m * 16 + 4 * tig); };
+      a[0] = row4(gid);
+      a[1] = row4(gid + 8);
+      a[2] = a[3] = 0u;  // k = 16 .. 31
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const int n = 8 * h + gid;
+        uint32_t v = 0;
+#pragma unroll
+        for (int i = 0; i < 4; i++) v |= (uint32_t)Bt[(4 * tig + i) * 16 + n] << (8 * i);
+        b[h][0] = v;
+        b[h][1] = 0u;
+      }
+    } else {
+      const uint16_t *At = static_cast<const uint16_t *>(A) + t * 256;
+      const uint16_t *Bt = static_cast<const uint16_t *>(B) + t * 256;
+      auto pair = [&](const uint16_t *p, int stride) { return (uint32_t)p[0] | ((uint32_t)p[stride] << 16); };
+      a[0] = pair(At + gid * 16 + 2 * tig, 1);
+      a[1] = pair(At + (gid + 8) * 16 + 2 * tig, 1);
+      a[2] = pair(At + gid * 16 + 2 * tig + 8, 1);
+      a[3] = pair(At + (gid + 8) * 16 + 2 * tig + 8, 1);
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const int n = 8 * h + gid;
+        b[h][0] = pair(Bt + (2 * tig) * 16 + n, 16);
+        b[h][1] = pair(Bt + (2 * tig + 8) * 16 + n, 16);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      const int col = 8 * h + 2 * tig;
+      float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4];
+      if (C != nullptr) {
+        const float *Ct = C + t * 256;
+        c[0] = Ct[gid * 16 + col];
+        c[1] = Ct[gid * 16 + col + 1];
+        c[2] = Ct[(gid + 8) * 16 + col];
+        c[3] = Ct[(gid + 8) * 16 + col + 1];
+      }
+      if constexpr (FMT == FMT_FP16) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%10,%11,%12,%13};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[h][0]), "r"(b[h][1]), "f"(c[0]), "f"(c[1]),
+              "f"(c[2]), "f"(c[3]));
+      } else if constexpr (FMT == FMT_BF16) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%10,%11,%12,%13};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[h][0]), "r"(b[h][1]), "f"(c[0]), "f"(c[1]),
+              "f"(c[2]), "f"(c[3]));
+      } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%10,%11,%12,%13};"
+            : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[h][0]), "r"(b[h][1]), "f"(c[0]), "f"(c[1]),
+              "f"(c[2]), "f"(c[3]));
+      }
+      float *Dt = D + t * 256;
+      Dt[gid * 16 + col] = d[0];
+      Dt[gid * 16 + col + 1] = d[1];
+      Dt[(gid + 8) * 16 + col] = d[2];
+      Dt[(gid + 8) * 16 + col + 1] = d[3];
+    }
+  }
+}
+
 }  // namespace mmaemu
 
 // ===========================================================================
@@ -1108,6 +1195,26 @@ int mmaemu_tiles(int model, int fmt, const void *A, const void *B, const float *
 #undef CALL_TILES
 }
 
+int mmaemu_native_tiles(int fmt, const void *A, const void *B, const float *C, float *D, size_t ntiles) {
+  if (fmt != MMAEMU_FP16 && fmt != MMAEMU_BF16 && fmt != MMAEMU_E4M3) return MMAEMU_EINVAL;
+  if (ntiles == 0) return MMAEMU_OK;
+  if (!A || !B || !D) return MMAEMU_EINVAL;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(D) || (C && !aligned16(C))) return MMAEMU_EINVAL;
+  if (ntiles > ((size_t)1 << 40)) return MMAEMU_EINVAL;
+  int sms = 0;
+  const int rc = check_device(&sms);
+  if (rc != MMAEMU_OK) return rc;
+  const size_t want = (ntiles + 7) / 8, cap = (size_t)sms * 8;
+  const unsigned blocks = (unsigned)(want < cap ? want : cap);
+  if (fmt == MMAEMU_FP16)
+    mmaemu::native_tiles_kernel<mmaemu::FMT_FP16><<<blocks, 256, 0, t_stream>>>(A, B, C, D, ntiles);
+  else if (fmt == MMAEMU_BF16)
+    mmaemu::native_tiles_kernel<mmaemu::FMT_BF16><<<blocks, 256, 0, t_stream>>>(A, B, C, D, ntiles);
+  else
+    mmaemu::native_tiles_kernel<mmaemu::FMT_E4M3><<<blocks, 256, 0, t_stream>>>(A, B, C, D, ntiles);
+  return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
+}
+
 int mmaemu_gemm(int model, int fmt, int M, int N, int K, const void *A, const void *B, const float *C, float *D,
                 uint32_t *fingerprint_out) {
   mmaemu::GemmParams p = row_major_params(M, N, K, A, B, C, D, fingerprint_out);
@@ -1177,7 +1284,9 @@ const char *mmaemu_strerror(int code) {
     case MMAEMU_EINVAL: return "invalid argument (enum, model/format pair, pointer, alignment or size)";
     case MMAEMU_ECUDA: return "CUDA runtime error";
     case MMAEMU_ETIMEOUT: return "bounded device wait expired";
-    case MMAEMU_EUNSUPPORTED: return "the current CUDA device is not an sm_100 (B200-class) GPU";
+    case MMAEMU_EUNSUPPORTED: return "unsupported: the current CUDA device is not an sm_100 (B200-class) GPU, "
+                                     "or the probe cannot be built for this format";
+    case MMAEMU_ECALLBACK: return "the MMA callback of a probe reported an error";
     default: return "unknown error code";
   }
 }

@@ -1,0 +1,326 @@
+// Probe API of libmmaemu (include/mmaemu_probe.h): the target tests and the
+// neutral-subgroup search of "Hawkeye: Reproducing GPU-Level
+// Non-Determinism (MLSys 2026)" (reading notes: "Target Tests" table;
+// Algorithm 4), run against any tile MMA given as a callback.  Host code
+// only; the built-in callbacks reach the GPU through the public C API.
+#include "mmaemu_probe.h"
+
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <vector>
+
+namespace {
+
+struct FmtInfo {
+  int p, bias, emin, emax, bytes;
+};
+
+bool fmt_info(int fmt, FmtInfo &f) {
+  switch (fmt) {
+    case MMAEMU_FP16: f = {10, 15, -14, 15, 2}; return true;
+    case MMAEMU_BF16: f = {7, 127, -126, 127, 2}; return true;
+    case MMAEMU_E4M3: f = {3, 7, -6, 8, 1}; return true;  // 2^8 is the largest power of two
+    default: return false;
+  }
+}
+
+// (-1)^s 2^e (1 + frac 2^-p), a normal value of the format
+uint32_t enc(const FmtInfo &f, int s, int e, uint32_t frac) {
+  const uint32_t field = (uint32_t)(e + f.bias);
+  return ((uint32_t)s << (8 * f.bytes - 1)) | (field << f.p) | frac;
+}
+uint32_t one(const FmtInfo &f) { return enc(f, 0, 0, 0); }
+uint32_t one_and_half(const FmtInfo &f, int s) { return enc(f, s, 0, 1u << (f.p - 1)); }
+
+// fp32 bit patterns
+uint32_t f32_pow2(int e) { return (uint32_t)(e + 127) << 23; }
+uint32_t f32_neg(uint32_t b) { return b ^ 0x80000000u; }
+
+// e = ea + eb with both in the format's normal exponent range
+bool split_exp(const FmtInfo &f, int e, int &ea, int &eb) {
+  ea = e >= 0 ? e / 2 : -((-e + 1) / 2);
+  if (ea < f.emin) ea = f.emin;
+  if (ea > f.emax) ea = f.emax;
+  eb = e - ea;
+  if (eb < f.emin) {
+    eb = f.emin;
+    ea = e - eb;
+  } else if (eb > f.emax) {
+    eb = f.emax;
+    ea = e - eb;
+  }
+  return ea >= f.emin && ea <= f.emax && eb >= f.emin && eb <= f.emax;
+}
+
+// A batch of probe instances, 16 per tile on the diagonal.
+struct Batch {
+  int fmt;
+  FmtInfo f;
+  size_t ntiles;
+  std::vector<uint8_t> A, B;
+  std::vector<uint32_t> C, D;
+
+  Batch(int fmt_, const FmtInfo &f_, size_t instances) : fmt(fmt_), f(f_) {
+    ntiles = (instances + 15) / 16;
+    A.assign(ntiles * 256 * f.bytes, 0);
+    B.assign(ntiles * 256 * f.bytes, 0);
+    C.assign(ntiles * 256, 0);
+    D.assign(ntiles * 256, 0);
+  }
+  void put(std::vector<uint8_t> &v, size_t elem, uint32_t bits) {
+    if (f.bytes == 1) {
+      v[elem] = (uint8_t)bits;
+    } else {
+      const uint16_t h = (uint16_t)bits;
+      std::memcpy(&v[2 * elem], &h, 2);
+    }
+  }
+  // product term k of instance q: A[i][k] = a, B[k][i] = b
+  void product(size_t q, int k, uint32_t a, uint32_t b) {
+    const size_t t = q / 16, i = q % 16;
+    put(A, t * 256 + i * 16 + k, a);
+    put(B, t * 256 + k * 16 + i, b);
+  }
+  void set_c(size_t q, uint32_t bits) { C[(q / 16) * 256 + (q % 16) * 17] = bits; }
+  uint32_t d(size_t q) const { return D[(q / 16) * 256 + (q % 16) * 17]; }
+  int run(mmaemu_mma_fn mma, void *ctx) {
+    return mma(ctx, fmt, A.data(), B.data(), C.data(), D.data(), ntiles) == 0 ? MMAEMU_OK : MMAEMU_ECALLBACK;
+  }
+};
+
+// exponent of C in the precision and alignment probes: products 2^(E0 - j)
+// for j up to 28 stay products of two normal values
+int probe_e0(int fmt) { return fmt == MMAEMU_FP16 ? 4 : fmt == MMAEMU_E4M3 ? 16 : 0; }
+
+constexpr int kMinJ = 16, kMaxJ = 27;
+
+int copy_run(int model_or_native, int fmt, const void *A, const void *B, const uint32_t *C, uint32_t *D,
+             size_t ntiles) {
+  FmtInfo f;
+  if (!fmt_info(fmt, f)) return MMAEMU_EINVAL;
+  const size_t in_bytes = ntiles * 256 * f.bytes, out_bytes = ntiles * 256 * 4;
+  void *dA = nullptr, *dB = nullptr, *dC = nullptr, *dD = nullptr;
+  int rc = MMAEMU_OK;
+  if (cudaMalloc(&dA, in_bytes) != cudaSuccess || cudaMalloc(&dB, in_bytes) != cudaSuccess ||
+      cudaMalloc(&dC, out_bytes) != cudaSuccess || cudaMalloc(&dD, out_bytes) != cudaSuccess)
+    rc = MMAEMU_ECUDA;
+  if (rc == MMAEMU_OK && (cudaMemcpy(dA, A, in_bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+                          cudaMemcpy(dB, B, in_bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+                          cudaMemcpy(dC, C, out_bytes, cudaMemcpyHostToDevice) != cudaSuccess))
+    rc = MMAEMU_ECUDA;
+  if (rc == MMAEMU_OK) {
+    rc = model_or_native < 0
+             ? mmaemu_native_tiles(fmt, dA, dB, static_cast<const float *>(dC), static_cast<float *>(dD), ntiles)
+             : mmaemu_tiles(model_or_native, fmt, dA, dB, static_cast<const float *>(dC), static_cast<float *>(dD),
+                            ntiles);
+  }
+  if (rc == MMAEMU_OK && cudaDeviceSynchronize() != cudaSuccess) rc = MMAEMU_ECUDA;
+  if (rc == MMAEMU_OK && cudaMemcpy(D, dD, out_bytes, cudaMemcpyDeviceToHost) != cudaSuccess) rc = MMAEMU_ECUDA;
+  cudaFree(dA);
+  cudaFree(dB);
+  cudaFree(dC);
+  cudaFree(dD);
+  return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mmaemu_mma_emulated(void *ctx, int fmt, const void *A, const void *B, const uint32_t *C, uint32_t *D,
+                        size_t ntiles) {
+  if (!ctx) return MMAEMU_EINVAL;
+  const int model = *static_cast<const int *>(ctx);
+  if (model != MMAEMU_AMPERE && model != MMAEMU_HOPPER) return MMAEMU_EINVAL;
+  return copy_run(model, fmt, A, B, C, D, ntiles);
+}
+
+int mmaemu_mma_native(void *, int fmt, const void *A, const void *B, const uint32_t *C, uint32_t *D,
+                      size_t ntiles) {
+  return copy_run(-1, fmt, A, B, C, D, ntiles);
+}
+
+int mmaemu_probe_precision(int fmt, mmaemu_mma_fn mma, void *ctx, int *fraction_bits) {
+  FmtInfo f;
+  if (!fmt_info(fmt, f) || !mma || !fraction_bits) return MMAEMU_EINVAL;
+  const int e0 = probe_e0(fmt), nj = kMaxJ - kMinJ + 1;
+  Batch b(fmt, f, nj + 1);
+  for (int q = 0; q <= nj; q++) b.set_c(q, f32_pow2(e0));
+  for (int q = 0; q < nj; q++) {
+    int ea, eb;
+    if (!split_exp(f, e0 - (kMinJ + q), ea, eb)) return MMAEMU_EINVAL;
+    for (int k = 0; k < 16; k++) b.product(q, k, enc(f, 0, ea, 0), enc(f, 0, eb, 0));
+  }
+  const int rc = b.run(mma, ctx);
+  if (rc != MMAEMU_OK) return rc;
+  // The terms are kept exactly iff D is the exact sum 2^E0 (1 + 2^(4 - j)),
+  // an fp32 value for j <= 27; a term off the grid gives C alone (dropped)
+  // or C plus 16 whole units (rounded up), never the exact sum.
+  int F = kMinJ - 1;
+  for (int q = 0; q < nj; q++) {
+    const int j = kMinJ + q;
+    const uint32_t exact = f32_pow2(e0) | (1u << (23 + 4 - j));
+    if (b.d(q) == exact) F = j;
+  }
+  *fraction_bits = F;
+  return MMAEMU_OK;
+}
+
+int mmaemu_probe_alignment_rounding(int fmt, mmaemu_mma_fn mma, void *ctx, int fraction_bits, int *mode) {
+  FmtInfo f;
+  if (!fmt_info(fmt, f) || !mma || !mode || fraction_bits < kMinJ - 1 || fraction_bits > kMaxJ)
+    return MMAEMU_EINVAL;
+  const int e0 = probe_e0(fmt);
+  int ea, eb;  // 1.5 2^(e0 - F - 1) = 0.75 units of the grid 2^(e0 - F)
+  if (!split_exp(f, e0 - fraction_bits - 1, ea, eb)) return MMAEMU_EINVAL;
+  Batch b(fmt, f, 3);
+  for (int q = 0; q < 3; q++) b.set_c(q, f32_pow2(e0));
+  for (int k = 0; k < 16; k++) {
+    b.product(0, k, enc(f, 0, ea, 1u << (f.p - 1)), enc(f, 0, eb, 0));
+    b.product(1, k, enc(f, 1, ea, 1u << (f.p - 1)), enc(f, 0, eb, 0));
+  }
+  const int rc = b.run(mma, ctx);
+  if (rc != MMAEMU_OK) return rc;
+  const bool up = b.d(0) != b.d(2), down = b.d(1) != b.d(2);
+  *mode = up ? (down ? MMAEMU_ROUND_NEAREST : MMAEMU_ROUND_UP) : (down ? MMAEMU_ROUND_DOWN : MMAEMU_ROUND_TOWARD_ZERO);
+  return MMAEMU_OK;
+}
+
+int mmaemu_probe_writeback_rounding(int fmt, mmaemu_mma_fn mma, void *ctx, int *mode) {
+  FmtInfo f;
+  if (!fmt_info(fmt, f) || !mma || !mode) return MMAEMU_EINVAL;
+  // Two exact sums per sign, each halfway between two fp32 values (ulp
+  // 2^-22 in [2, 4)): 3.5 - 2^-23 (even neighbour above in magnitude) and
+  // 3.5 - 3 2^-23 (even neighbour below).  C = 2 - 2^-23 or 2 - 3 2^-23,
+  // one product 1.5, both of either sign.  The product is the last term
+  // (k = 15), so an earlier accumulation stage only carries C, which it
+  // holds exactly, and the tie reaches the final cast.
+  const uint32_t c_bits[2] = {0x3FFFFFFFu, 0x3FFFFFFDu};
+  const uint32_t lower[2] = {0x405FFFFFu, 0x405FFFFEu};  // magnitudes rounded down
+  Batch b(fmt, f, 4);
+  for (int q = 0; q < 4; q++) {
+    const int neg = q >> 1;
+    b.set_c(q, c_bits[q & 1] | ((uint32_t)neg << 31));
+    b.product(q, 15, one_and_half(f, neg), one(f));
+  }
+  const int rc = b.run(mma, ctx);
+  if (rc != MMAEMU_OK) return rc;
+  int up[2][2];  // [sign][case]: magnitude rounded up (1), down (0), neither (-1)
+  for (int q = 0; q < 4; q++) {
+    const uint32_t mag = b.d(q) & 0x7FFFFFFFu, sign = b.d(q) >> 31, lo = lower[q & 1];
+    up[q >> 1][q & 1] = sign != (uint32_t)(q >> 1) ? -1 : mag == lo ? 0 : mag == lo + 1 ? 1 : -1;
+  }
+  auto is = [&](int p0, int p1, int n0, int n1) {
+    return up[0][0] == p0 && up[0][1] == p1 && up[1][0] == n0 && up[1][1] == n1;
+  };
+  if (is(0, 0, 0, 0)) *mode = MMAEMU_ROUND_TOWARD_ZERO;
+  else if (is(1, 0, 1, 0)) *mode = MMAEMU_ROUND_NEAREST_EVEN;
+  else if (is(1, 1, 1, 1)) *mode = MMAEMU_ROUND_NEAREST_AWAY;
+  else if (is(1, 1, 0, 0)) *mode = MMAEMU_ROUND_UP;
+  else if (is(0, 0, 1, 1)) *mode = MMAEMU_ROUND_DOWN;
+  else *mode = MMAEMU_ROUND_OTHER;
+  return MMAEMU_OK;
+}
+
+int mmaemu_probe_normalization(int fmt, mmaemu_mma_fn mma, void *ctx, int fraction_bits, int *delayed) {
+  FmtInfo f;
+  if (!fmt_info(fmt, f) || !mma || !delayed || fraction_bits < 23 || fraction_bits > kMaxJ)
+    return MMAEMU_EINVAL;
+  Batch b(fmt, f, 2);
+  const uint32_t c_plain = f32_pow2(23 - fraction_bits);
+  b.set_c(0, c_plain | 1u);  // one more bit, 2^-F
+  b.set_c(1, c_plain);
+  for (int q = 0; q < 2; q++) {
+    b.product(q, 0, one_and_half(f, 0), one_and_half(f, 0));  // +2.25 at exponent 0
+    b.product(q, 1, one_and_half(f, 1), one_and_half(f, 0));  // -2.25
+  }
+  const int rc = b.run(mma, ctx);
+  if (rc != MMAEMU_OK) return rc;
+  // the products cancel, so delayed normalisation returns C exactly; with
+  // the products normalised first C's last bit is half a unit of the grid
+  // and is dropped or rounded to a whole unit -- never returned exactly
+  *delayed = b.d(0) == (c_plain | 1u) && b.d(1) == c_plain ? 1 : 0;
+  return MMAEMU_OK;
+}
+
+int mmaemu_probe_subnormal(int fmt, mmaemu_mma_fn mma, void *ctx, int fraction_bits, int *renormalized) {
+  FmtInfo f;
+  if (!fmt_info(fmt, f) || !mma || !renormalized || fraction_bits < kMinJ - 1 || fraction_bits > kMaxJ)
+    return MMAEMU_EINVAL;
+  // C = a quarter unit of the grid 2^(emin - F) that the product sets when
+  // it keeps the minimum exponent emin (dropped by truncation and by
+  // rounding to nearest alike), and a whole multiple of the grid
+  // 2^(emin - p - F) it sets when renormalised.  The sum must be exact in
+  // fp32: F + 2 - p <= 23.
+  const int gap = fraction_bits + 2 - f.p;
+  if (fmt == MMAEMU_BF16 || gap > 23) return MMAEMU_EUNSUPPORTED;
+  Batch b(fmt, f, 2);
+  const uint32_t min_sub = 1u;  // field 0, fraction 1
+  for (int q = 0; q < 2; q++) b.product(q, 0, min_sub, one(f));
+  b.set_c(0, f32_pow2(f.emin - fraction_bits - 2));
+  const int rc = b.run(mma, ctx);
+  if (rc != MMAEMU_OK) return rc;
+  const uint32_t product = f32_pow2(f.emin - f.p);  // 2^(emin - p), the product's value
+  *renormalized = b.d(0) == (product | (1u << (23 - gap))) && b.d(1) == product ? 1 : 0;
+  return MMAEMU_OK;
+}
+
+int mmaemu_probe_neutral(int fmt, mmaemu_mma_fn mma, void *ctx, const uint32_t *subsets, size_t nsubsets,
+                         uint8_t *neutral) {
+  FmtInfo f;
+  if (!fmt_info(fmt, f) || !mma || (nsubsets && (!subsets || !neutral))) return MMAEMU_EINVAL;
+  if (nsubsets == 0) return MMAEMU_OK;
+  if (nsubsets > ((size_t)1 << 24)) return MMAEMU_EINVAL;
+  for (size_t s = 0; s < nsubsets; s++) {
+    const uint32_t m = subsets[s];
+    const int size = __builtin_popcount(m);
+    if ((m >> 17) != 0 || size < 2 || size > 16) return MMAEMU_EINVAL;
+  }
+  // +-X and small terms per format.  Every small term, and C's 2^-20 bit,
+  // has a bit below the grid 2^(16 - F) of a group whose maximum is X's
+  // exponent 16 (so a group holding X truncates it, for any F <= 29) and
+  // above the grid 2^-F set by C = 1 (so it is kept otherwise):
+  //   FP16: small_i = (1 + (2i-1) 2^-10)(1 + 2^-10), lowest bit 2^-20
+  //   BF16: small_i = (1 + (2i-1) 2^-7) 2^-8 (1 + 2^-7), lowest bit 2^-22
+  //   E4M3: small_i = 2^-6 (1 + f/8) 2^-6 (1 + 1/8), f odd, lowest bit 2^-18
+  const uint32_t xa = enc(f, 0, 8, 0), c_base = 0x3F800008u;  // X = 256 x 256; C = 1 + 2^-20
+  const float x_value = 65536.0f;
+  const uint32_t small_b = fmt == MMAEMU_E4M3 ? enc(f, 0, -6, 1) : enc(f, 0, 0, 1);
+  auto small_a = [&](int i) {  // term i = 1 .. 16
+    if (fmt == MMAEMU_E4M3) return enc(f, 0, -6, (uint32_t)(2 * ((i - 1) & 3) + 1));
+    if (fmt == MMAEMU_BF16) return enc(f, 0, -8, (uint32_t)(2 * i - 1));
+    return enc(f, 0, 0, (uint32_t)(2 * i - 1));
+  };
+  uint32_t c_pos, c_neg;
+  std::memcpy(&c_pos, &x_value, 4);
+  c_neg = f32_neg(c_pos);
+  const uint32_t xa_neg = xa | (1u << (8 * f.bytes - 1));
+
+  Batch b(fmt, f, 2 * nsubsets);
+  for (size_t s = 0; s < nsubsets; s++) {
+    const uint32_t m = subsets[s];
+    const int first = __builtin_ctz(m), last = 31 - __builtin_clz(m);
+    for (int zeroed = 0; zeroed < 2; zeroed++) {
+      const size_t q = 2 * s + zeroed;
+      for (int i = 0; i < 17; i++) {
+        const bool in = (m >> i) & 1u;
+        int sign = 0;  // +1 / -1 for the engineered +-X, 0 for a zero term
+        if (in && !zeroed) sign = i == first ? 1 : i == last ? -1 : 0;
+        if (i == 0) {
+          b.set_c(q, in ? (sign > 0 ? c_pos : sign < 0 ? c_neg : 0u) : c_base);
+        } else if (!in) {
+          b.product(q, i - 1, small_a(i), small_b);
+        } else if (sign != 0) {
+          b.product(q, i - 1, sign > 0 ? xa : xa_neg, xa);
+        }
+      }
+    }
+  }
+  const int rc = b.run(mma, ctx);
+  if (rc != MMAEMU_OK) return rc;
+  for (size_t s = 0; s < nsubsets; s++) neutral[s] = b.d(2 * s) == b.d(2 * s + 1) ? 1 : 0;
+  return MMAEMU_OK;
+}
+
+}  // extern "C"

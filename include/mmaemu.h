@@ -56,6 +56,7 @@ enum { MMAEMU_FP16 = 0, MMAEMU_BF16 = 1, MMAEMU_E4M3 = 2 };
 #define MMAEMU_ECUDA (-2)        /* a CUDA runtime call or launch failed                    */
 #define MMAEMU_ETIMEOUT (-3)     /* a bounded device wait gave up (reserved; no call waits) */
 #define MMAEMU_EUNSUPPORTED (-4) /* the current device is not an sm_100 GPU                 */
+#define MMAEMU_ECALLBACK (-5)    /* a probe's MMA callback failed (mmaemu_probe.h)           */
 
 /* Select the CUDA stream (a cudaStream_t passed as void*) that the calling
  * host thread's later calls enqueue on; NULL selects the legacy default

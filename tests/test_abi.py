@@ -12,7 +12,10 @@ HEADER = os.path.join(ROOT, "include", "mmaemu.h")
 
 
 def header_text():
-    return open(HEADER).read()
+    """All of include/*.h (the C ABI: mmaemu.h and mmaemu_probe.h)."""
+    import glob
+
+    return "\n".join(open(h).read() for h in sorted(glob.glob(os.path.join(os.path.dirname(HEADER), "*.h"))))
 
 
 def declared_functions():
@@ -41,8 +44,11 @@ def L():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == ["mmaemu_gemm", "mmaemu_gemm_strided_batched", "mmaemu_gemm_verify",
-                                    "mmaemu_set_stream", "mmaemu_strerror", "mmaemu_tiles", "mmaemu_xorsum",
-                                    "mmaemu_xorsum_noalloc"]
+                                    "mmaemu_mma_emulated", "mmaemu_mma_native", "mmaemu_native_tiles",
+                                    "mmaemu_probe_alignment_rounding", "mmaemu_probe_neutral",
+                                    "mmaemu_probe_normalization", "mmaemu_probe_precision", "mmaemu_probe_subnormal",
+                                    "mmaemu_probe_writeback_rounding", "mmaemu_set_stream", "mmaemu_strerror",
+                                    "mmaemu_tiles", "mmaemu_xorsum", "mmaemu_xorsum_noalloc"]
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -59,11 +65,15 @@ def test_constants_match_python_binding():
     assert c["MMAEMU_FP16"] == m.FORMATS["fp16"] and c["MMAEMU_BF16"] == m.FORMATS["bf16"]
     assert c["MMAEMU_E4M3"] == m.FORMATS["e4m3"]
     assert (c["MMAEMU_OK"], c["MMAEMU_EINVAL"], c["MMAEMU_ECUDA"], c["MMAEMU_ETIMEOUT"],
-            c["MMAEMU_EUNSUPPORTED"]) == (0, -1, -2, -3, -4)
+            c["MMAEMU_EUNSUPPORTED"], c["MMAEMU_ECALLBACK"]) == (0, -1, -2, -3, -4, -5)
+    from bit_exact_tensor_b200 import probe
+
+    for code, name in probe.ROUNDING.items():
+        assert c["MMAEMU_ROUND_" + name.upper().replace("-", "_")] == code
 
 
 def test_strerror_and_set_stream(L):
-    for code in (0, -1, -2, -3, -4, 7):
+    for code in (0, -1, -2, -3, -4, -5, 7):
         assert L.mmaemu_strerror(code)
     assert L.mmaemu_set_stream(None) == 0
 

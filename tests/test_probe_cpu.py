@@ -1,0 +1,138 @@
+"""The probe API (include/mmaemu_probe.h) on the CPU: the library's target
+tests and neutral-subgroup search run against MMA callbacks built from the
+oracle -- the two models, planted-mistake variants of the model and what-if
+models -- and must recover exactly what each callback computes.
+
+Page: "Hawkeye: Reproducing GPU-Level Non-Determinism (MLSys 2026)" (reading
+notes): "Target Tests" table, Algorithm 4, Obs. 2 and Obs. 3.
+"""
+
+import numpy as np
+import pytest
+
+import oracle.mma_model as mm
+from oracle import cref
+from test_oracle_mutations import MUTANTS, _mutant
+
+PAIRS = (("ampere", "fp16"), ("ampere", "bf16"), ("hopper", "fp16"), ("hopper", "bf16"), ("hopper", "e4m3"))
+
+
+@pytest.fixture(scope="module")
+def probe():
+    from bit_exact_tensor_b200 import _build
+    from bit_exact_tensor_b200 import probe as p
+
+    _build.build_library()
+    return p
+
+
+def oracle_target(probe, model):
+    return probe.from_callable(lambda fmt, A, B, C: cref.tiles(model, fmt, A, B, C, nthreads=4), f"oracle {model}")
+
+
+def diagonal_target(probe, module, model_obj, name):
+    """An MMA that evaluates only the diagonal outputs with a Python model
+    (the probes read nothing else)."""
+
+    def f(fmt, A, B, C):
+        fm = module.FORMATS[fmt]
+        D = np.zeros(C.shape, dtype=np.uint32)
+        for t in range(A.shape[0]):
+            for i in range(16):
+                D[t, i, i] = module.mma_element(model_obj, fm, [int(x) for x in A[t, i, :]],
+                                                [int(x) for x in B[t, :, i]], int(C[t, i, i]))
+        return D
+
+    return probe.from_callable(f, name)
+
+
+@pytest.mark.parametrize("model,fmt", PAIRS)
+def test_probes_recover_both_models_exhaustively(probe, model, fmt):
+    """Obs. 2 and 3: Ampere keeps 23 fraction bits (24-bit significand),
+    Hopper 24; truncating alignment, toward-zero write-back, delayed
+    normalisation, subnormal products kept at the minimum exponent; the only
+    nontrivial neutral subgroup over all 2^17 subsets is {C, P[1..8]} for
+    Ampere and there is none for Hopper."""
+    r = probe.characterize(oracle_target(probe, model), fmt, exhaustive=True)
+    assert r["fraction_bits"] == (23 if model == "ampere" else 24)
+    assert r["alignment_rounding"] == "toward-zero"
+    assert r["writeback_rounding"] == "toward-zero"
+    assert r["normalization"] == "delayed"
+    assert r["subnormal_products"] == (None if fmt == "bf16" else "not renormalized")
+    assert r["neutral_subgroups"] == ([tuple(range(9))] if model == "ampere" else [])
+
+
+# (mutant name, model, probe key, value the probe must report)
+DETECT = [
+    ("alignment rounds to nearest", "ampere", "alignment_rounding", "nearest"),
+    ("alignment floors the signed value", "ampere", "alignment_rounding", "down"),
+    ("products normalised before accumulation", "ampere", "normalization", "normalized first"),
+    ("subnormal operands renormalised", "hopper", "subnormal_products", "renormalized"),
+    ("Ampere accumulates in one stage", "ampere", "neutral_subgroups", []),
+    ("Ampere stage boundary off by one", "ampere", "neutral_subgroups", [tuple(range(10))]),
+    ("Hopper keeps 24 bits, not 25", "hopper", "fraction_bits", 23),
+    ("Ampere keeps 25 bits", "ampere", "fraction_bits", 24),
+    ("write-back rounds to nearest", "ampere", "writeback_rounding", "nearest-away"),
+]
+
+
+@pytest.mark.parametrize("name,model,key,want", DETECT, ids=[d[0] for d in DETECT])
+def test_probe_reports_the_planted_difference(probe, name, model, key, want):
+    import sys
+
+    orig, repl = next((o, r) for n, o, r in MUTANTS if n == name)
+    mod = _mutant(orig, repl)
+    try:
+        t = diagonal_target(probe, mod, getattr(mod, model.upper()), name)
+        r = probe.characterize(t, "fp16", exhaustive=False)
+    finally:
+        sys.modules.pop("mma_model_mutant", None)
+    assert r[key] == want, r
+    # everything not planted still reads as the model
+    base = {"fraction_bits": 23 if model == "ampere" else 24, "alignment_rounding": "toward-zero",
+            "writeback_rounding": "toward-zero", "normalization": "delayed",
+            "subnormal_products": "not renormalized",
+            "neutral_subgroups": [tuple(range(9))] if model == "ampere" else []}
+    for k, v in base.items():
+        if k != key and not (key == "fraction_bits" and k == "neutral_subgroups"):
+            assert r[k] == v, (k, r)
+
+
+@pytest.mark.parametrize("F,groups,want_neutral", [
+    (26, (tuple(range(0, 8)), tuple(range(8, 16))), [tuple(range(9))]),
+    (25, (tuple(range(0, 16)),), []),
+    # every prefix {C, P1..Pk} ending at a stage boundary cancels invisibly
+    (23, (tuple(range(0, 4)), tuple(range(4, 8)), tuple(range(8, 12)), tuple(range(12, 16))),
+     [tuple(range(5)), tuple(range(9)), tuple(range(13))]),
+    (24, (tuple(range(0, 12)), tuple(range(12, 16))), [tuple(range(13))]),
+])
+def test_probe_recovers_what_if_models(probe, F, groups, want_neutral):
+    """Models the pages do not describe -- other widths and stage splits --
+    are recovered too (the probes do not assume the two known answers)."""
+    model = mm.Model("what-if", F, groups)
+    r = probe.characterize(diagonal_target(probe, mm, model, "what-if"), "fp16", exhaustive=False)
+    assert r["fraction_bits"] == F
+    assert r["alignment_rounding"] == "toward-zero" and r["writeback_rounding"] == "toward-zero"
+    assert r["neutral_subgroups"] == want_neutral
+
+
+def test_probe_argument_errors(probe):
+    import ctypes
+
+    from bit_exact_tensor_b200 import MmaEmuError
+
+    t = oracle_target(probe, "hopper")
+    with pytest.raises(MmaEmuError):
+        probe.alignment_rounding(t, "fp16", 40)  # fraction bits outside the probe's range
+    with pytest.raises(MmaEmuError):
+        probe.neutral_subgroups(t, "fp16", [(3,)])  # a single term cannot cancel
+    assert probe.subnormal_products(t, "bf16", 24) is None
+
+    def failing(fmt, A, B, C):
+        raise RuntimeError("the MMA is unavailable")
+
+    with pytest.raises(MmaEmuError) as e:
+        probe.precision(probe.from_callable(failing), "fp16")
+    assert e.value.code == -5
+    L = probe._lib()
+    assert L.mmaemu_probe_precision(7, probe.native().fn, None, ctypes.byref(ctypes.c_int())) == -1

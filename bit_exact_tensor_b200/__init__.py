@@ -18,7 +18,7 @@ import threading
 __all__ = ["MODELS", "FORMATS", "MmaEmuError", "lib", "tiles", "gemm", "gemm_verify", "gemm_batched", "xorsum",
            "xorsum_noalloc", "gemm_host", "set_stream", "NO_MISMATCH"]
 
-MODELS = {"ampere": 0, "hopper": 1}
+MODELS = {"ampere": 0, "hopper": 1, "b200": 2, "lovelace": 0}
 FORMATS = {"fp16": 0, "bf16": 1, "e4m3": 2}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))

@@ -132,7 +132,7 @@ int mmaemu_mma_emulated(void *ctx, int fmt, const void *A, const void *B, const 
                         size_t ntiles) {
   if (!ctx) return MMAEMU_EINVAL;
   const int model = *static_cast<const int *>(ctx);
-  if (model != MMAEMU_AMPERE && model != MMAEMU_HOPPER) return MMAEMU_EINVAL;
+  if (model != MMAEMU_AMPERE && model != MMAEMU_HOPPER && model != MMAEMU_B200) return MMAEMU_EINVAL;
   return copy_run(model, fmt, A, B, C, D, ntiles);
 }
 

@@ -19,7 +19,7 @@ import numpy as np
 
 FORMAT_BITS = {"fp16": (5, 10, 15), "bf16": (8, 7, 127), "e4m3": (4, 3, 7)}
 PAIRS = (("ampere", "fp16"), ("ampere", "bf16"), ("hopper", "fp16"), ("hopper", "bf16"),
-         ("hopper", "e4m3"))
+         ("hopper", "e4m3"), ("b200", "fp16"), ("b200", "bf16"))
 
 
 def in_dtype(fmt: str):

@@ -21,7 +21,7 @@ _SRC = os.path.join(_HERE, "mmaemu_ref.c")
 _BUILD = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_BUILD, "liborc.so")
 
-MODEL = {"ampere": 0, "hopper": 1}
+MODEL = {"ampere": 0, "hopper": 1, "b200": 2}
 FMT = {"fp16": 0, "bf16": 1, "e4m3": 2}
 IN_DTYPE = {"fp16": np.uint16, "bf16": np.uint16, "e4m3": np.uint8}
 

@@ -259,6 +259,8 @@ def rational_expect(model: str, fmt: str, A, B, c) -> int:
                            emin_in=_FMT_EMIN[fmt], emin_c=-126,
                            a_negzero=[x == sign_bit for x in A], b_negzero=[x == sign_bit for x in B],
                            c_negzero=c == 0x80000000)
+    if res[0] == "nan":
+        return M.nan  # the model's NaN pattern (0x7FC00000 for both models on the pages)
     if res[0] == "fin":
         res = rm.round_rz(res[1], 23, -126, 127)
     return rm.encode_fp32(res)

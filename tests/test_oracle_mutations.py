@@ -83,8 +83,8 @@ MUTANTS = [
      "    assert q < (1 << out.p)\n    return sign_bit | q",
      "    return sign_bit"),
     ("Inf x 0 not NaN",
-     "            if ak.is_zero or bk.is_zero:\n                return _nan(out)",
-     "            if False:\n                return _nan(out)"),
+     "            if ak.is_zero or bk.is_zero:\n                return _nan(out, model)",
+     "            if False:\n                return _nan(out, model)"),
     ("zero terms take part in the max exponent",
      "nz = [t for t in terms if t.A != 0]",
      "nz = list(terms)\n    if not any(t.A for t in nz):\n        return None"),

@@ -83,7 +83,8 @@ def test_invalid_arguments_rejected_before_any_device_work(L):
     buf = ctypes.create_string_buffer(4096 + 16)
     p = (ctypes.addressof(buf) + 15) & ~15
     # bad enums, Ampere x E4M3, bad shapes, NULL and misaligned pointers
-    assert L.mmaemu_gemm(2, 0, 16, 16, 16, p, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(3, 0, 16, 16, 16, p, p, None, p, None) == EINVAL
+    assert L.mmaemu_gemm(2, 2, 16, 16, 16, p, p, None, p, None) == EINVAL  # B200 x E4M3 is not modelled
     assert L.mmaemu_gemm(0, 3, 16, 16, 16, p, p, None, p, None) == EINVAL
     assert L.mmaemu_gemm(0, 2, 16, 16, 16, p, p, None, p, None) == EINVAL
     assert L.mmaemu_gemm(1, 0, 16, 24, 16, p, p, None, p, None) == EINVAL

@@ -123,6 +123,49 @@ int mmaemu_probe_subnormal(int fmt, mmaemu_mma_fn mma, void *ctx, int fraction_b
 int mmaemu_probe_neutral(int fmt, mmaemu_mma_fn mma, void *ctx, const uint32_t *subsets, size_t nsubsets,
                          uint8_t *neutral);
 
+/* Exponent threshold (the BF16 paragraph of the recovered pipeline: "max
+ * exponent threshold -133").  For a candidate floor L, one instance sums
+ * (2^k - 2) units of 2^(L - F) (k = F - L - 149, so 2^k units make
+ * 2^-149) and fifteen products of 0.875 units: with the group maximum
+ * floored at L or above, the small products truncate away and the result is
+ * +0; with a lower floor (or none) they carry the sum to 2^-149.  L runs
+ * over F - 158 .. F - 150 (-133 is always inside).  *e_floor = the largest L
+ * that gives +0; MMAEMU_NO_FLOOR if none does (no floor at or above
+ * F - 158); F - 150 if all do (a lower bound).  BF16 only (other formats'
+ * products cannot reach the threshold): MMAEMU_EUNSUPPORTED otherwise.     */
+#define MMAEMU_NO_FLOOR (-100000)
+int mmaemu_probe_floor(int fmt, mmaemu_mma_fn mma, void *ctx, int fraction_bits, int *e_floor);
+
+/* A model as data: what the target tests measure, and what the emulation
+ * needs ("Hawkeye: Reproducing GPU-Level Non-Determinism (MLSys 2026)"
+ * reading notes -- Obs. 2 and 3 for the fields; the BF16 paragraph for the
+ * threshold).                                                              */
+#define MMAEMU_FLOOR_ANY 100000 /* in an identify query: the floor was not measured */
+typedef struct mmaemu_model_desc {
+  int fraction_bits;          /* F: bits kept below the group's largest exponent  */
+  int stages;                 /* accumulation stages (C joins the first)          */
+  int stage_products[4];      /* products per stage, in k order; they sum to 16   */
+  int e_floor;                /* floor on each group's max exponent, NO_FLOOR,   */
+                              /* or (in a query) FLOOR_ANY                        */
+  int alignment_rounding;     /* MMAEMU_ROUND_*                                   */
+  int writeback_rounding;     /* MMAEMU_ROUND_*                                   */
+  int delayed_normalization;  /* 1: products accumulate unnormalised              */
+  int subnormal_renormalized; /* 1: subnormal products are renormalised           */
+  uint32_t nan_bits;          /* fp32 NaN result pattern; 0 in a query: any       */
+} mmaemu_model_desc;
+
+/* The parameters of a built-in model (MMAEMU_AMPERE, _HOPPER, _B200;
+ * MMAEMU_LOVELACE is Ampere).  Errors: MMAEMU_EINVAL.                     */
+int mmaemu_model_describe(int model, mmaemu_model_desc *out);
+
+/* The built-in model with exactly these parameters (nan_bits 0 matches any
+ * NaN pattern, e_floor FLOOR_ANY any floor; stage_products beyond `stages`
+ * are ignored) -- e.g. the
+ * result of the target tests on some MMA.  MMAEMU_EUNSUPPORTED when no
+ * built-in model matches: the library can describe that MMA but not
+ * emulate it.  Errors: MMAEMU_EINVAL.                                      */
+int mmaemu_model_identify(const mmaemu_model_desc *desc, int *model);
+
 #ifdef __cplusplus
 }
 #endif

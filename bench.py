@@ -52,21 +52,22 @@ WORKLOAD = "gemm M=N=K=4096, Ampere FP16 model, fp32 C=0 and D, fused per-16x16-
 # DRAM bytes per launch of the GEMM kernel (dram__bytes_read.sum + dram__bytes_write.sum)
 # from one ncu capture (profiles/gemm_ampere_fp16_4096_ncu_full.md), valid only
 # for the kernel sources it was taken on, identified by their hash.
-TRAFFIC_CAPTURE = {"source_sha16": "681427d6e1eecd29", "bytes": 194_845_696}
+TRAFFIC_CAPTURE = {"source_sha16": "6439321e1f16f36d", "bytes": 194_486_016}
 KERNEL_SOURCES = ("bit_exact_tensor_b200/csrc/mmaemu.cu", "bit_exact_tensor_b200/csrc/mmaemu_core.cuh",
                   "include/mmaemu.h")
 
 
 HBM_PEAK_GBS = 6557.4  # measured copy bandwidth on this machine's B200s (MEASURED_PEAKS.json)
 DEFAULT_WORKLOAD = "gemm-ampere-fp16-4096"
-PAIRS = (("ampere", "fp16"), ("ampere", "bf16"), ("hopper", "fp16"), ("hopper", "bf16"), ("hopper", "e4m3"))
+PAIRS = (("ampere", "fp16"), ("ampere", "bf16"), ("hopper", "fp16"), ("hopper", "bf16"), ("hopper", "e4m3"),
+         ("b200", "fp16"), ("b200", "bf16"))
 E4M3_LAYER = "gemm-hopper-e4m3-8192x4096x14336"
 # variants of the E4M3 layer GEMM: fingerprints only (no D written), verify
 # a claimed D instead of storing it, weights stored [N][K] (B transposed)
 GEMM_MODES = ("fponly", "verify", "wt")
 BATCHED = "gemm-batched-ampere-fp16-8x1024x4096x4096"
 WORKLOAD_NAMES = ({DEFAULT_WORKLOAD, "gemm-hopper-bf16-4096", "gemm-hopper-bf16-4096-wide", E4M3_LAYER,
-                   "tiles-ampere-fp16-4096", BATCHED}
+                   "tiles-ampere-fp16-4096", BATCHED, "gemm-b200-fp16-4096"}
                   | {f"{E4M3_LAYER}-{m}" for m in GEMM_MODES}
                   | {f"tiles-{m}-{f}-100k" for m, f in PAIRS})
 
@@ -113,6 +114,10 @@ def workload_spec(name: str) -> dict:
         return spec
     if name == DEFAULT_WORKLOAD:
         return gemm("ampere", "fp16", lambda r: wl.config3(seed=3 + 1000 * r), M, N, K, WORKLOAD)
+    if name == "gemm-b200-fp16-4096":
+        return gemm("b200", "fp16", lambda r: wl.config3(seed=3 + 1000 * r), 4096, 4096, 4096,
+                    "gemm M=N=K=4096, B200 FP16 model (B200's own MMA, measured), A, B ~ N(0,1), C = 0, "
+                    "fused per-tile xorsum")
     if name == "gemm-hopper-bf16-4096":
         return gemm("hopper", "bf16", lambda r: wl.config4(seed=4 + 1000 * r), 4096, 4096, 4096,
                     "gemm M=N=K=4096, Hopper BF16 model, log2|x| ~ U[-60, 60], fused per-tile xorsum")
@@ -130,7 +135,9 @@ def workload_spec(name: str) -> dict:
             def make(r, f=f):
                 A_, B_, C_, _ = wl.config2(f, seed=1 + 1000 * r)
                 return A_, B_, C_
-            return tiles(m, f, make, 100_000, f"100,000 random + adversarial tiles, {m.capitalize()} {f.upper()} model")
+            return tiles(m, f, make, 100_000,
+                         f"100,000 random + adversarial tiles, {m.capitalize() if m != 'b200' else 'B200'} "
+                         f"{f.upper()} model")
     raise ValueError(name)
 
 

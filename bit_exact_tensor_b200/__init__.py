@@ -16,7 +16,7 @@ import os
 import threading
 
 __all__ = ["MODELS", "FORMATS", "MmaEmuError", "lib", "tiles", "gemm", "gemm_verify", "gemm_batched", "xorsum",
-           "xorsum_noalloc", "gemm_host", "set_stream", "NO_MISMATCH"]
+           "xorsum_noalloc", "gemm_host", "set_stream", "trim_workspace", "NO_MISMATCH"]
 
 MODELS = {"ampere": 0, "hopper": 1, "b200": 2, "lovelace": 0}
 FORMATS = {"fp16": 0, "bf16": 1, "e4m3": 2}
@@ -345,3 +345,9 @@ def xorsum_noalloc(t) -> int:
 
 
 NOALLOC_MAX_WORDS = 1 << 27  # MMAEMU_XORSUM_NOALLOC_MAX_WORDS
+
+
+def trim_workspace():
+    """Return the current device's cached GEMM workspace (the decoded
+    operands of earlier calls) to the device."""
+    _check(lib().mmaemu_trim_workspace(), "mmaemu_trim_workspace")

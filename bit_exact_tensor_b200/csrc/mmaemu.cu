@@ -15,6 +15,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "mmaemu.h"
 #include "mmaemu_core.cuh"
@@ -778,50 +779,140 @@ struct GemmParams {
   int M, N, K, ta, tb;
   long long lda, ldb, ldc, ldd, ldr;
   long long sA, sB, sC, sD, sR, sF;
+  // decoded operand panels (workspace written by the decode pass): for each
+  // batch entry, 64-row block of A or 128-column block of B, and K chunk, a
+  // blob laid out exactly like that part of a shared-memory panel; and one
+  // special-value flag word per blob (A blobs' flags first)
+  unsigned char *dA, *dB;
+  uint32_t *flags;
+  int batch;
 };
+
+// Decoded panel blobs: the A part (aM, aN, aP, aN2) and the B part (bM, bN,
+// bP, bN2) of a GPanel, stored contiguously in that order.
+constexpr size_t ABLOB = offsetof(GPanel, bM), BBLOB = sizeof(GPanel) - offsetof(GPanel, bM);
+static_assert(ABLOB == 16384 && BBLOB == 28672, "panel layout");
+static_assert(offsetof(GPanel, aN) == 4096 && offsetof(GPanel, aP) == 8192 && offsetof(GPanel, aN2) == 12288 &&
+                  offsetof(GPanel, bN) - ABLOB == 8192 && offsetof(GPanel, bP) - ABLOB == 16384 &&
+                  offsetof(GPanel, bN2) - ABLOB == 24576,
+              "blob field offsets");
+
+// Decode pass, A side: one thread per 8 k-consecutive elements (row m,
+// chunk j, half h) into the blob of (batch entry, m / 64, j).
+template <int MODEL, int FMT>
+__global__ void __launch_bounds__(256) decode_a_kernel(const GemmParams p) {
+  constexpr int ESIZE = FMT == FMT_E4M3 ? 1 : 2;
+  constexpr int SH = ModelT<MODEL>::F - 2 * FmtT<FMT>::P;
+  const int nrb = (p.M + GBM - 1) / GBM, nch = p.K / 16;
+  const int m = blockIdx.x * blockDim.x + threadIdx.x;
+  if (m >= nrb * GBM) return;
+  const int j = blockIdx.y >> 1, h = blockIdx.y & 1;
+  const size_t bz = blockIdx.z;
+  const void *A = static_cast<const unsigned char *>(p.A) + bz * (size_t)p.sA * ESIZE;
+  const bool valid = m < p.M;
+  const size_t k = 16 * (size_t)j + 8 * h, lda = (size_t)p.lda;
+  const Raw8<FMT> raw = !p.ta ? load_row8<FMT>(A, (size_t)m * lda + k, valid) : load_col8<FMT>(A, k * lda + m, lda, valid);
+  const int rb = m / GBM, ml = m % GBM;
+  unsigned char *blob = p.dA + ((bz * nrb + rb) * nch + j) * ABLOB;
+  uint32_t special = 0;
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    const Dec d = decode<FMT>(raw.get(i));
+    const size_t off = (size_t)(8 * h + i) * GBM * 4 + (size_t)ml * 4;
+    *reinterpret_cast<uint32_t *>(blob + 0 * 4096 + off) = d.m << SH;
+    *reinterpret_cast<int32_t *>(blob + 1 * 4096 + off) = d.n;
+    *reinterpret_cast<int32_t *>(blob + 2 * 4096 + off) = (int32_t)(d.s | 1u);
+    *reinterpret_cast<uint32_t *>(blob + 3 * 4096 + off) = pack16(d.n, d.n);
+    special |= d.special;
+  }
+  if (special) atomicOr(&p.flags[(bz * nrb + rb) * nch + j], 1u);
+}
+
+// Decode pass, B side: one thread per 8 k-consecutive elements of column n.
+template <int MODEL, int FMT>
+__global__ void __launch_bounds__(256) decode_b_kernel(const GemmParams p) {
+  constexpr int ESIZE = FMT == FMT_E4M3 ? 1 : 2;
+  const int nrb = (p.M + GBM - 1) / GBM, ncb = (p.N + GBN - 1) / GBN, nch = p.K / 16;
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= ncb * GBN) return;
+  const int j = blockIdx.y >> 1, h = blockIdx.y & 1;
+  const size_t bz = blockIdx.z;
+  const void *B = static_cast<const unsigned char *>(p.B) + bz * (size_t)p.sB * ESIZE;
+  const bool valid = n < p.N;
+  const size_t k = 16 * (size_t)j + 8 * h, ldb = (size_t)p.ldb;
+  const Raw8<FMT> raw = !p.tb ? load_col8<FMT>(B, k * ldb + n, ldb, valid) : load_row8<FMT>(B, (size_t)n * ldb + k, valid);
+  const int cb = n / GBN, nl = n % GBN;
+  unsigned char *blob = p.dB + ((bz * ncb + cb) * nch + j) * BBLOB;
+  uint32_t special = 0;
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    const Dec d = decode<FMT>(raw.get(i));
+    const size_t kk = (size_t)(8 * h + i), off = kk * GBN * 4 + (size_t)nl * 4;
+    *reinterpret_cast<uint32_t *>(blob + 0 * 8192 + off) = d.m;
+    *reinterpret_cast<int32_t *>(blob + 1 * 8192 + off) = d.n;
+    *reinterpret_cast<int32_t *>(blob + 2 * 8192 + off) = (int32_t)(d.s | 1u);
+    *reinterpret_cast<int16_t *>(blob + 3 * 8192 + kk * GBN * 2 + (size_t)nl * 2) = (int16_t)d.n;
+    special |= d.special;
+  }
+  if (special) atomicOr(&p.flags[(size_t)p.batch * nrb * nch + (bz * ncb + cb) * nch + j], 1u);
+}
+
+// 16-byte asynchronous global -> shared copy
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Blocks are visited in groups of GROUP_ROWS row blocks, column block by
+// column block, so that the blocks resident at one time share A and B
+// panels and the decoded operands are reused from L2.
+constexpr int GROUP_ROWS = 16;
 
 template <int MODEL, int FMT>
 __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const GemmParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   GPanel *panels = reinterpret_cast<GPanel *>(smem_raw);
-  constexpr int ESIZE = FMT == FMT_E4M3 ? 1 : 2;
   const int M = p.M, N = p.N, K = p.K;
   const size_t bz = blockIdx.z;
-  const void *A = static_cast<const unsigned char *>(p.A) + bz * (size_t)p.sA * ESIZE;
-  const void *B = static_cast<const unsigned char *>(p.B) + bz * (size_t)p.sB * ESIZE;
-  const size_t lda = (size_t)p.lda, ldb = (size_t)p.ldb;
+
+  // grouped block order (row block rb, column block cb)
+  const int nrb = gridDim.y, ncb = gridDim.x;
+  const int lin = blockIdx.y * ncb + blockIdx.x, per_group = GROUP_ROWS * ncb;
+  const int g = lin / per_group, rem = lin - g * per_group, first = g * GROUP_ROWS;
+  const int rows = min(GROUP_ROWS, nrb - first);
+  const int rb = first + rem % rows, cb = rem / rows;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int row0 = blockIdx.y * GBM, col0 = blockIdx.x * GBN;
+  const int row0 = rb * GBM, col0 = cb * GBN;
   // this thread's 4 x 8 outputs
   const int rl = (warp >> 2) * 32 + (lane >> 2) * GR;
   const int cl = (warp & 3) * 32 + (lane & 3) * GCC;
   const bool out_valid = (row0 + rl < M) && (col0 + cl < N);
 
-  // loader roles: A row am / half ah (threads < 128); B column bn / half bh
-  const int am = tid & (GBM - 1), ah = (tid >> 6) & 1;
-  const bool a_loader = tid < 2 * GBM;
-  const bool a_valid = a_loader && (row0 + am < M);
-  const int bn = tid & (GBN - 1), bh = tid >> 7;
-  const bool b_valid = col0 + bn < N;
-
+  // Per chunk, the block copies its decoded A and B blobs (16 KiB + 28 KiB)
+  // into the panel with 16-byte asynchronous copies: 4 + 7 per thread.
   const int nchunks = K / 16;
-  Raw8<FMT> ra, rb;
-  // 8 k-consecutive elements: one vector load where k is the contiguous
-  // index, else 8 loads that are coalesced across the loader threads
-  auto load_chunk = [&](int j) {
-    const size_t k = 16 * (size_t)j;
-    if (!p.ta) ra = load_row8<FMT>(A, (size_t)(row0 + am) * lda + k + 8 * ah, a_valid);
-    else ra = load_col8<FMT>(A, (k + 8 * ah) * lda + row0 + am, lda, a_valid);
-    if (!p.tb) rb = load_col8<FMT>(B, (k + 8 * bh) * ldb + col0 + bn, ldb, b_valid);
-    else rb = load_row8<FMT>(B, (size_t)(col0 + bn) * ldb + k + 8 * bh, b_valid);
+  const unsigned char *blob_a = p.dA + (bz * nrb + rb) * (size_t)nchunks * ABLOB;
+  const unsigned char *blob_b = p.dB + (bz * ncb + cb) * (size_t)nchunks * BBLOB;
+  const uint32_t *flag_a = p.flags + (bz * nrb + rb) * (size_t)nchunks;
+  const uint32_t *flag_b = p.flags + (size_t)p.batch * nrb * nchunks + (bz * ncb + cb) * (size_t)nchunks;
+  auto issue_chunk = [&](int j, GPanel &P) {
+    const uint4 *sa = reinterpret_cast<const uint4 *>(blob_a + (size_t)j * ABLOB);
+    const uint4 *sb = reinterpret_cast<const uint4 *>(blob_b + (size_t)j * BBLOB);
+    uint4 *da = reinterpret_cast<uint4 *>(&P);
+    uint4 *db = reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(&P) + ABLOB);
+#pragma unroll
+    for (int i = 0; i < (int)(ABLOB / 16 / GTHREADS); i++) cp_async16(da + tid + i * GTHREADS, sa + tid + i * GTHREADS);
+#pragma unroll
+    for (int i = 0; i < (int)(BBLOB / 16 / GTHREADS); i++) cp_async16(db + tid + i * GTHREADS, sb + tid + i * GTHREADS);
+    cp_async_commit();
   };
-  auto store_chunk = [&](GPanel &P) -> uint32_t {
-    uint32_t sp = 0;
-    if (a_loader) sp |= store_a8<MODEL, FMT>(P, am, ah, ra);
-    sp |= store_b8<FMT>(P, bn, bh, rb);
-    return sp;
-  };
+  static_assert(ABLOB % (16 * GTHREADS) == 0 && BBLOB % (16 * GTHREADS) == 0, "copies per thread");
 
   // accumulator: fp32 bits V on the float-assisted path (FP16 / E4M3 while
   // the values stay in its range), else the integer state (n, X) in V's place
@@ -834,10 +925,16 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const Gemm
   if (!kFloatAssisted<FMT>) fast = false;
   if (!fast) values_to_state<GR, GCC>(Np, V);
 
-  load_chunk(0);
-  bool panel_special = __syncthreads_or(store_chunk(panels[0])) != 0;
+  issue_chunk(0, panels[0]);
+  cp_async_wait_all();
+  __syncthreads();
+  bool panel_special = (flag_a[0] | flag_b[0]) != 0;
   for (int j = 0; j < nchunks; j++) {
-    if (j + 1 < nchunks) load_chunk(j + 1);
+    bool next_special = false;
+    if (j + 1 < nchunks) {
+      issue_chunk(j + 1, panels[(j + 1) & 1]);
+      next_special = (flag_a[j + 1] | flag_b[j + 1]) != 0;
+    }
     if constexpr (kFloatAssisted<FMT>) {
       if (fast) {
         bool to_integer = false;
@@ -852,7 +949,11 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const Gemm
     } else {
       mma_chunk<MODEL, FMT, GR, GCC>(panels[j & 1], rl, cl, Np, X, dneg0, panel_special);
     }
-    if (j + 1 < nchunks) panel_special = __syncthreads_or(store_chunk(panels[(j + 1) & 1])) != 0;
+    if (j + 1 < nchunks) {
+      cp_async_wait_all();
+      __syncthreads();
+      panel_special = next_special;
+    }
   }
 
   // epilogue: store D, compare with the claimed D, per-16x16-tile xorsum
@@ -1143,6 +1244,34 @@ int check_device(int *sms = nullptr) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Library-private stream-ordered memory pool per device for the GEMM's
+// decoded-operand workspace.  Freed workspace stays in the pool (release
+// threshold: unlimited) so that repeated GEMMs reuse it without new
+// device allocations; mmaemu_trim_workspace returns it.
+std::mutex g_pool_mutex;
+cudaMemPool_t g_pool[kMaxDevices] = {};
+
+cudaMemPool_t workspace_pool() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_pool_mutex);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+    uint64_t threshold = UINT64_MAX;
+    if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &threshold) != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return nullptr;
+    }
+    g_pool[dev] = pool;
+  }
+  return g_pool[dev];
+}
+
 bool valid_pair(int model, int fmt) {
   if (model != MMAEMU_AMPERE && model != MMAEMU_HOPPER && model != MMAEMU_B200) return false;
   if (fmt != MMAEMU_FP16 && fmt != MMAEMU_BF16 && fmt != MMAEMU_E4M3) return false;
@@ -1162,14 +1291,41 @@ bool valid_pair(int model, int fmt) {
   } while (0)
 
 template <int MODEL, int FMT>
-int launch_gemm(const mmaemu::GemmParams &p, int batch) {
+int launch_gemm(const mmaemu::GemmParams &p_in, int batch) {
+  using mmaemu::ABLOB;
+  using mmaemu::BBLOB;
+  mmaemu::GemmParams p = p_in;
+  const int nrb = (p.M + mmaemu::GBM - 1) / mmaemu::GBM, ncb = (p.N + mmaemu::GBN - 1) / mmaemu::GBN;
+  const int nch = p.K / 16;
+  // workspace: decoded blobs and their flags, stream-ordered, released
+  // after the GEMM
+  const size_t a_bytes = (size_t)batch * nrb * nch * ABLOB, b_bytes = (size_t)batch * ncb * nch * BBLOB;
+  const size_t f_bytes = (size_t)batch * (nrb + ncb) * nch * sizeof(uint32_t);
+  unsigned char *ws = nullptr;
+  cudaMemPool_t pool = workspace_pool();
+  if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), a_bytes + b_bytes + f_bytes, pool,
+                                       t_stream) != cudaSuccess)
+    return MMAEMU_ECUDA;
+  p.dA = ws;
+  p.dB = ws + a_bytes;
+  p.flags = reinterpret_cast<uint32_t *>(ws + a_bytes + b_bytes);
+  p.batch = batch;
+  int rc = MMAEMU_OK;
   const size_t smem = 2 * sizeof(mmaemu::GPanel);
   auto kern = mmaemu::gemm_kernel<MODEL, FMT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return MMAEMU_ECUDA;
-  dim3 grid((p.N + mmaemu::GBN - 1) / mmaemu::GBN, (p.M + mmaemu::GBM - 1) / mmaemu::GBM, batch);
-  kern<<<grid, mmaemu::GTHREADS, smem, t_stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
+  if (cudaMemsetAsync(p.flags, 0, f_bytes, t_stream) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    rc = MMAEMU_ECUDA;
+  if (rc == MMAEMU_OK) {
+    const dim3 ga((nrb * mmaemu::GBM + 255) / 256, 2 * nch, batch), gb((ncb * mmaemu::GBN + 255) / 256, 2 * nch, batch);
+    mmaemu::decode_a_kernel<MODEL, FMT><<<ga, 256, 0, t_stream>>>(p);
+    mmaemu::decode_b_kernel<MODEL, FMT><<<gb, 256, 0, t_stream>>>(p);
+    dim3 grid(ncb, nrb, batch);
+    kern<<<grid, mmaemu::GTHREADS, smem, t_stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) rc = MMAEMU_ECUDA;
+  }
+  if (cudaFreeAsync(ws, t_stream) != cudaSuccess) rc = MMAEMU_ECUDA;
+  return rc;
 }
 
 // Shape, layout and alignment rules shared by the GEMM entry points.
@@ -1177,6 +1333,7 @@ int validate_gemm(const mmaemu::GemmParams &p, long long batch) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0 || (p.M & 15) || (p.N & 15) || (p.K & 15)) return MMAEMU_EINVAL;
   if (batch < 1 || batch > 65535) return MMAEMU_EINVAL;
   if ((long long)p.M / mmaemu::GBM >= 65535) return MMAEMU_EINVAL;
+  if ((long long)p.K / 16 * 2 > 65535) return MMAEMU_EINVAL;  // decode-pass grid
   if (!p.A || !p.B) return MMAEMU_EINVAL;
   if (!p.D && !p.fp && !p.Dref) return MMAEMU_EINVAL;  // nothing to produce
   if (p.Dref && !p.mism) return MMAEMU_EINVAL;
@@ -1349,6 +1506,15 @@ int mmaemu_xorsum(const void *D, size_t n, uint32_t *out_host) {
   if (cudaStreamSynchronize(t_stream) != cudaSuccess) rc = MMAEMU_ECUDA;
   if (rc == MMAEMU_OK) *out_host = result;
   return rc;
+}
+
+int mmaemu_trim_workspace(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MMAEMU_ECUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MMAEMU_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_pool_mutex);
+  if (g_pool[dev] && cudaMemPoolTrimTo(g_pool[dev], 0) != cudaSuccess) return MMAEMU_ECUDA;
+  return MMAEMU_OK;
 }
 
 const char *mmaemu_strerror(int code) {

@@ -84,13 +84,23 @@ int mmaemu_set_stream(void *cuda_stream);
 int mmaemu_tiles(int model, int fmt, const void *A, const void *B, const float *C, float *D,
                  size_t ntiles);
 
+/* GEMM implementation note (all three GEMM calls): each call first decodes
+ * A and B once into panel form, then the MMA kernel copies those panels
+ * instead of decoding per output block.  The decoded operands live in a
+ * stream-ordered workspace of
+ *   batch * K/16 * (ceil(M/64) * 16 KiB + ceil(N/128) * 28 KiB + small)
+ * bytes (about 500 MB for M = N = K = 4096) taken from a memory pool owned
+ * by the library.  Freed workspace stays in that pool for the next call;
+ * mmaemu_trim_workspace hands it back to the device.  A failed workspace
+ * allocation returns MMAEMU_ECUDA before anything is enqueued.            */
+
 /* Large MatMul composed of 16x16x16 tiles (Obs. 4): D = C + A . B where K is
  * walked in 16-wide chunks in ascending order and the fp32 result of each
  * chunk is the C of the next, so every output element is
  *   d_0 = C[m][n];  d_{j+1} = MMA16(A[m][16j..16j+15], B[16j..16j+15][n], d_j).
  *   A: [M][K] in fmt; B: [K][N] in fmt; C, D: [M][N] fp32; C may be NULL (+0)
  *   and may equal D (in place); no other overlap.
- *   M, N, K: positive multiples of 16; M / 64 below 65535.
+ *   M, N, K: positive multiples of 16; M / 64 below 65535; K / 8 at most 65535.
  *   fingerprint_out: NULL, or [(M/16)*(N/16)] uint32 written with the
  *   xorsum (XOR of the 256 fp32 bit patterns) of each 16x16 tile of D, tiles
  *   in row-major tile-grid order -- the AEGIS xorsum fingerprint, fused into
@@ -179,6 +189,11 @@ int mmaemu_xorsum(const void *D, size_t n, uint32_t *out_host);
  *   MMAEMU_EUNSUPPORTED.                                                    */
 #define MMAEMU_XORSUM_NOALLOC_MAX_WORDS ((size_t)1 << 27)
 int mmaemu_xorsum_noalloc(const void *D, size_t n, uint32_t *out_host);
+
+/* Return the current device's unused GEMM workspace (see above) to the
+ * device.  Workspace still in use by enqueued GEMMs is kept.  Errors:
+ * MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED.                                       */
+int mmaemu_trim_workspace(void);
 
 /* Static message for a return code. */
 const char *mmaemu_strerror(int code);

@@ -49,7 +49,8 @@ def test_header_declares_the_boundary():
                                     "mmaemu_probe_alignment_rounding", "mmaemu_probe_floor", "mmaemu_probe_neutral",
                                     "mmaemu_probe_normalization", "mmaemu_probe_precision", "mmaemu_probe_subnormal",
                                     "mmaemu_probe_writeback_rounding", "mmaemu_set_stream", "mmaemu_strerror",
-                                    "mmaemu_tiles", "mmaemu_xorsum", "mmaemu_xorsum_noalloc"]
+                                    "mmaemu_tiles", "mmaemu_trim_workspace", "mmaemu_xorsum",
+                                    "mmaemu_xorsum_noalloc"]
 
 
 def test_library_exports_every_declared_symbol(L):

@@ -151,6 +151,26 @@ def test_worst_case_magnitudes_in_the_k_chain(cref, model, fmt):
     assert np.array_equal(D, want), first_mismatch(D, want)
 
 
+def test_workspace_reuse_and_trim(cref):
+    """GEMMs of different sizes share the library's cached workspace; after
+    trimming it the next call allocates afresh; results never change."""
+    import torch
+
+    import bit_exact_tensor_b200 as mmaemu
+
+    A, B, C = normal_inputs(208, 272, 160, "fp16", seed=8)
+    want = cref.gemm("hopper", "fp16", A, B, C)
+    for shape in ((208, 272, 160), (64, 128, 32), (208, 272, 160)):
+        M, N, K = shape
+        D, _ = run_gemm("hopper", "fp16", A[:M, :K].copy(), B[:K, :N].copy(), C[:M, :N].copy())
+        assert np.array_equal(D, cref.gemm("hopper", "fp16", A[:M, :K].copy(), B[:K, :N].copy(),
+                                           C[:M, :N].copy()))
+    mmaemu.trim_workspace()
+    torch.cuda.synchronize()
+    D, _ = run_gemm("hopper", "fp16", A, B, C)
+    assert np.array_equal(D, want)
+
+
 def test_null_c_in_place_and_no_fingerprint(cref):
     import bit_exact_tensor_b200 as mmaemu
 

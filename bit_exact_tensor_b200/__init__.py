@@ -299,22 +299,37 @@ def xorsum(t) -> int:
     return int(res.value)
 
 
-def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bool = True, device="cuda"):
-    """End-to-end call from host memory: copies A, B (and C) to the device,
-    runs the emulated GEMM and copies D (and fingerprints) back.  Host
-    tensors should be pinned for full-speed copies.  Returns CPU tensors."""
+def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bool = True, device=None):
+    """End-to-end call from host memory (mmaemu_gemm_host): host A, B (and C)
+    in, host D and fingerprints out, with the transfers overlapped with the
+    arithmetic inside the library.  Host tensors should be page-locked
+    (``tensor.pin_memory()``) for the overlap.  ``device`` selects the CUDA
+    device (default: the current one).  Returns CPU tensors (D, fp)."""
     torch = _torch()
-    A = A_host.to(device, non_blocking=True)
-    B = B_host.to(device, non_blocking=True)
-    C = C_host.to(device, non_blocking=True) if C_host is not None else None
-    D, fp = gemm(model, fmt, A, B, C, fingerprint=fingerprint)
-    D_host = torch.empty(D.shape, dtype=D.dtype, pin_memory=True)
-    D_host.copy_(D, non_blocking=True)
-    fp_host = None
-    if fp is not None:
-        fp_host = torch.empty(fp.shape, dtype=fp.dtype, pin_memory=True)
-        fp_host.copy_(fp, non_blocking=True)
-    torch.cuda.current_stream().synchronize()
+    mi, fi = _model_fmt(model, fmt)
+    for t, name in ((A_host, "A"), (B_host, "B")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CPU tensor")
+        if t.dtype not in _in_dtypes()[fmt]:
+            raise TypeError(f"{name} has dtype {t.dtype}, expected one of {_in_dtypes()[fmt]} for {fmt}")
+    if A_host.dim() != 2 or B_host.dim() != 2 or A_host.shape[1] != B_host.shape[0]:
+        raise ValueError("A must be [M,K] and B [K,N]")
+    M, K = A_host.shape
+    N = B_host.shape[1]
+    if C_host is not None:
+        if C_host.is_cuda or not C_host.is_contiguous() or tuple(C_host.shape) != (M, N) or \
+                C_host.dtype not in (torch.float32, torch.int32, torch.uint32):
+            raise TypeError("C must be a contiguous CPU fp32 tensor [M,N]")
+    D_host = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
+    fp_host = torch.empty(((M // 16) * (N // 16),), dtype=torch.int32, pin_memory=True) if fingerprint else None
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        set_stream()
+        fn = lib().mmaemu_gemm_host
+        fn.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 5
+        fn.restype = ctypes.c_int
+        _check(fn(mi, fi, M, N, K, A_host.data_ptr(), B_host.data_ptr(),
+                  C_host.data_ptr() if C_host is not None else None, D_host.data_ptr(),
+                  fp_host.data_ptr() if fp_host is not None else None), "mmaemu_gemm_host")
     return D_host, fp_host
 
 

@@ -789,9 +789,9 @@ struct GemmParams {
   // decoded operand panels (workspace written by the decode pass): for each
   // batch entry, 64-row block of A or 128-column block of B, and K chunk, a
   // blob laid out exactly like that part of a shared-memory panel; and one
-  // special-value flag word per blob (A blobs' flags first)
+  // special-value flag word per blob
   unsigned char *dA, *dB;
-  uint32_t *flags;
+  uint32_t *flags_a, *flags_b;
   int batch;
 };
 
@@ -832,14 +832,14 @@ __global__ void __launch_bounds__(256) decode_a_kernel(const GemmParams p) {
     *reinterpret_cast<uint32_t *>(blob + 3 * 4096 + off) = pack16(d.n, d.n);
     special |= d.special;
   }
-  if (special) atomicOr(&p.flags[(bz * nrb + rb) * nch + j], 1u);
+  if (special) atomicOr(&p.flags_a[(bz * nrb + rb) * nch + j], 1u);
 }
 
 // Decode pass, B side: one thread per 8 k-consecutive elements of column n.
 template <int MODEL, int FMT>
 __global__ void __launch_bounds__(256) decode_b_kernel(const GemmParams p) {
   constexpr int ESIZE = FMT == FMT_E4M3 ? 1 : 2;
-  const int nrb = (p.M + GBM - 1) / GBM, ncb = (p.N + GBN - 1) / GBN, nch = p.K / 16;
+  const int ncb = (p.N + GBN - 1) / GBN, nch = p.K / 16;
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= ncb * GBN) return;
   const int j = blockIdx.y >> 1, h = blockIdx.y & 1;
@@ -861,7 +861,7 @@ __global__ void __launch_bounds__(256) decode_b_kernel(const GemmParams p) {
     *reinterpret_cast<int16_t *>(blob + 3 * 8192 + kk * GBN * 2 + (size_t)nl * 2) = (int16_t)d.n;
     special |= d.special;
   }
-  if (special) atomicOr(&p.flags[(size_t)p.batch * nrb * nch + (bz * ncb + cb) * nch + j], 1u);
+  if (special) atomicOr(&p.flags_b[(bz * ncb + cb) * nch + j], 1u);
 }
 
 // 16-byte asynchronous global -> shared copy
@@ -906,8 +906,8 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const Gemm
   const int nchunks = K / 16;
   const unsigned char *blob_a = p.dA + (bz * nrb + rb) * (size_t)nchunks * ABLOB;
   const unsigned char *blob_b = p.dB + (bz * ncb + cb) * (size_t)nchunks * BBLOB;
-  const uint32_t *flag_a = p.flags + (bz * nrb + rb) * (size_t)nchunks;
-  const uint32_t *flag_b = p.flags + (size_t)p.batch * nrb * nchunks + (bz * ncb + cb) * (size_t)nchunks;
+  const uint32_t *flag_a = p.flags_a + (bz * nrb + rb) * (size_t)nchunks;
+  const uint32_t *flag_b = p.flags_b + (bz * ncb + cb) * (size_t)nchunks;
   auto issue_chunk = [&](int j, GPanel &P) {
     const uint4 *sa = reinterpret_cast<const uint4 *>(blob_a + (size_t)j * ABLOB);
     const uint4 *sb = reinterpret_cast<const uint4 *>(blob_b + (size_t)j * BBLOB);
@@ -1297,41 +1297,201 @@ bool valid_pair(int model, int fmt) {
     return MMAEMU_EINVAL;                                                               \
   } while (0)
 
+// Workspace sizes of one GEMM (all batch entries): decoded A and B blobs
+// and their flag words.
+struct GemmSizes {
+  int nrb, ncb, nch;
+  size_t a_bytes, b_bytes, fa_bytes, fb_bytes;
+};
+GemmSizes gemm_sizes(int M, int N, int K, int batch) {
+  GemmSizes z;
+  z.nrb = (M + mmaemu::GBM - 1) / mmaemu::GBM;
+  z.ncb = (N + mmaemu::GBN - 1) / mmaemu::GBN;
+  z.nch = K / 16;
+  z.a_bytes = (size_t)batch * z.nrb * z.nch * mmaemu::ABLOB;
+  z.b_bytes = (size_t)batch * z.ncb * z.nch * mmaemu::BBLOB;
+  z.fa_bytes = (size_t)batch * z.nrb * z.nch * sizeof(uint32_t);
+  z.fb_bytes = (size_t)batch * z.ncb * z.nch * sizeof(uint32_t);
+  return z;
+}
+
+// Decode pass for B (p.dB, p.flags_b set) on `stream`.
 template <int MODEL, int FMT>
-int launch_gemm(const mmaemu::GemmParams &p_in, int batch) {
-  using mmaemu::ABLOB;
-  using mmaemu::BBLOB;
-  mmaemu::GemmParams p = p_in;
-  const int nrb = (p.M + mmaemu::GBM - 1) / mmaemu::GBM, ncb = (p.N + mmaemu::GBN - 1) / mmaemu::GBN;
-  const int nch = p.K / 16;
-  // workspace: decoded blobs and their flags, stream-ordered, released
-  // after the GEMM
-  const size_t a_bytes = (size_t)batch * nrb * nch * ABLOB, b_bytes = (size_t)batch * ncb * nch * BBLOB;
-  const size_t f_bytes = (size_t)batch * (nrb + ncb) * nch * sizeof(uint32_t);
-  unsigned char *ws = nullptr;
-  cudaMemPool_t pool = workspace_pool();
-  if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), a_bytes + b_bytes + f_bytes, pool,
-                                       t_stream) != cudaSuccess)
-    return MMAEMU_ECUDA;
-  p.dA = ws;
-  p.dB = ws + a_bytes;
-  p.flags = reinterpret_cast<uint32_t *>(ws + a_bytes + b_bytes);
-  p.batch = batch;
-  int rc = MMAEMU_OK;
+int launch_decode_b(const mmaemu::GemmParams &p, int batch, cudaStream_t stream) {
+  const GemmSizes z = gemm_sizes(p.M, p.N, p.K, batch);
+  if (cudaMemsetAsync(p.flags_b, 0, z.fb_bytes, stream) != cudaSuccess) return MMAEMU_ECUDA;
+  const dim3 gb((z.ncb * mmaemu::GBN + 255) / 256, 2 * z.nch, batch);
+  mmaemu::decode_b_kernel<MODEL, FMT><<<gb, 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
+}
+
+// Decode pass for A and the MMA kernel (B already decoded) on `stream`.
+template <int MODEL, int FMT>
+int launch_decode_a_gemm(const mmaemu::GemmParams &p, int batch, cudaStream_t stream) {
+  const GemmSizes z = gemm_sizes(p.M, p.N, p.K, batch);
   const size_t smem = 2 * sizeof(mmaemu::GPanel);
   auto kern = mmaemu::gemm_kernel<MODEL, FMT>;
-  if (cudaMemsetAsync(p.flags, 0, f_bytes, t_stream) != cudaSuccess ||
+  if (cudaMemsetAsync(p.flags_a, 0, z.fa_bytes, stream) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    rc = MMAEMU_ECUDA;
-  if (rc == MMAEMU_OK) {
-    const dim3 ga((nrb * mmaemu::GBM + 255) / 256, 2 * nch, batch), gb((ncb * mmaemu::GBN + 255) / 256, 2 * nch, batch);
-    mmaemu::decode_a_kernel<MODEL, FMT><<<ga, 256, 0, t_stream>>>(p);
-    mmaemu::decode_b_kernel<MODEL, FMT><<<gb, 256, 0, t_stream>>>(p);
-    dim3 grid(ncb, nrb, batch);
-    kern<<<grid, mmaemu::GTHREADS, smem, t_stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) rc = MMAEMU_ECUDA;
-  }
+    return MMAEMU_ECUDA;
+  const dim3 ga((z.nrb * mmaemu::GBM + 255) / 256, 2 * z.nch, batch);
+  mmaemu::decode_a_kernel<MODEL, FMT><<<ga, 256, 0, stream>>>(p);
+  kern<<<dim3(z.ncb, z.nrb, batch), mmaemu::GTHREADS, smem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
+}
+
+template <int MODEL, int FMT>
+int launch_gemm(const mmaemu::GemmParams &p_in, int batch) {
+  mmaemu::GemmParams p = p_in;
+  const GemmSizes z = gemm_sizes(p.M, p.N, p.K, batch);
+  // workspace: decoded blobs and their flags, stream-ordered, released
+  // after the GEMM
+  unsigned char *ws = nullptr;
+  cudaMemPool_t pool = workspace_pool();
+  if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws),
+                                       z.a_bytes + z.b_bytes + z.fa_bytes + z.fb_bytes, pool, t_stream) != cudaSuccess)
+    return MMAEMU_ECUDA;
+  p.dA = ws;
+  p.dB = ws + z.a_bytes;
+  p.flags_a = reinterpret_cast<uint32_t *>(ws + z.a_bytes + z.b_bytes);
+  p.flags_b = reinterpret_cast<uint32_t *>(ws + z.a_bytes + z.b_bytes + z.fa_bytes);
+  p.batch = batch;
+  int rc = launch_decode_b<MODEL, FMT>(p, batch, t_stream);
+  if (rc == MMAEMU_OK) rc = launch_decode_a_gemm<MODEL, FMT>(p, batch, t_stream);
   if (cudaFreeAsync(ws, t_stream) != cudaSuccess) rc = MMAEMU_ECUDA;
+  return rc;
+}
+
+mmaemu::GemmParams row_major_params(int M, int N, int K, const void *A, const void *B, const float *C, float *D,
+                                    uint32_t *fp) {
+  mmaemu::GemmParams p{};
+  p.A = A; p.B = B; p.C = C; p.D = D; p.fp = fp;
+  p.M = M; p.N = N; p.K = K;
+  p.lda = K; p.ldb = N; p.ldc = N; p.ldd = N; p.ldr = N;
+  return p;
+}
+
+// Library-owned streams per device for mmaemu_gemm_host: copies in, copies
+// out, and a second compute stream.
+cudaStream_t g_copy_in[kMaxDevices] = {}, g_copy_out[kMaxDevices] = {}, g_compute2[kMaxDevices] = {};
+
+int host_streams(cudaStream_t &in, cudaStream_t &out, cudaStream_t &compute2) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MMAEMU_ECUDA;
+  std::lock_guard<std::mutex> lock(g_pool_mutex);
+  for (cudaStream_t *st : {&g_copy_in[dev], &g_copy_out[dev], &g_compute2[dev]})
+    if (!*st && cudaStreamCreateWithFlags(st, cudaStreamNonBlocking) != cudaSuccess) return MMAEMU_ECUDA;
+  in = g_copy_in[dev];
+  out = g_copy_out[dev];
+  compute2 = g_compute2[dev];
+  return MMAEMU_OK;
+}
+
+// mmaemu_gemm from host memory: B is copied and decoded once; A and C go in
+// row slabs (a multiple of 64 rows) on a copy stream while earlier slabs
+// compute, alternately on the caller's stream and a second compute stream
+// (so that one slab's last partial wave of blocks overlaps the next slab),
+// and each slab's D (and fingerprints) returns on another copy stream as
+// soon as that slab is done.
+template <int MODEL, int FMT>
+int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, const float *C_h, float *D_h,
+                     uint32_t *fp_h) {
+  constexpr size_t ES = FMT == mmaemu::FMT_E4M3 ? 1 : 2;
+  cudaStream_t s_in, s_out, c2;
+  int rc = host_streams(s_in, s_out, c2);
+  if (rc != MMAEMU_OK) return rc;
+  const cudaStream_t cs[2] = {t_stream, c2};
+  const int rows_per = ((M + 7) / 8 + mmaemu::GBM - 1) / mmaemu::GBM * mmaemu::GBM;
+  const int nslab = (M + rows_per - 1) / rows_per;
+  const GemmSizes zs = gemm_sizes(rows_per, N, K, 1), zb = gemm_sizes(M, N, K, 1);
+  const size_t a_bytes = (size_t)M * K * ES, b_bytes = (size_t)K * N * ES, cd_bytes = (size_t)M * N * 4;
+  const size_t fp_bytes = fp_h ? (size_t)(M / 16) * (N / 16) * 4 : 0;
+  // device buffers, each 256-byte aligned inside one pool allocation
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t o_b = up(a_bytes), o_c = o_b + up(b_bytes), o_d = o_c + (C_h ? up(cd_bytes) : 0);
+  // two A-blob workspaces and flag arrays, one per compute stream
+  const size_t o_fp = o_d + up(cd_bytes), o_wa = o_fp + up(fp_bytes), o_wb = o_wa + 2 * up(zs.a_bytes);
+  const size_t o_fa = o_wb + up(zb.b_bytes), o_fb = o_fa + 2 * up(zs.fa_bytes), total = o_fb + up(zb.fb_bytes);
+  unsigned char *buf = nullptr;
+  cudaMemPool_t pool = workspace_pool();
+  if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void **>(&buf), total, pool, t_stream) != cudaSuccess)
+    return MMAEMU_ECUDA;
+  unsigned char *dA = buf, *dB = buf + o_b;
+  float *dC = C_h ? reinterpret_cast<float *>(buf + o_c) : nullptr;
+  float *dD = reinterpret_cast<float *>(buf + o_d);
+  uint32_t *dfp = fp_h ? reinterpret_cast<uint32_t *>(buf + o_fp) : nullptr;
+
+  const int nev = 2 + 2 * nslab + 3;
+  cudaEvent_t ev[2 + 2 * 8 + 3];
+  int made = 0;
+  for (; made < nev; made++)
+    if (cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming) != cudaSuccess) {
+      rc = MMAEMU_ECUDA;
+      break;
+    }
+  cudaEvent_t &e_alloc = ev[0], &e_b = ev[1], &e_out = ev[nev - 1], &e_bdec = ev[nev - 2], &e_c2 = ev[nev - 3];
+  auto e_in = [&](int sl) -> cudaEvent_t & { return ev[2 + sl]; };
+  auto e_done = [&](int sl) -> cudaEvent_t & { return ev[2 + nslab + sl]; };
+  auto ok = [&](cudaError_t e) {
+    if (e != cudaSuccess) rc = MMAEMU_ECUDA;
+    return rc == MMAEMU_OK;
+  };
+  if (rc == MMAEMU_OK && ok(cudaEventRecord(e_alloc, t_stream)) && ok(cudaStreamWaitEvent(s_in, e_alloc, 0)) &&
+      ok(cudaStreamWaitEvent(s_out, e_alloc, 0)) && ok(cudaStreamWaitEvent(c2, e_alloc, 0)) &&
+      ok(cudaMemcpyAsync(dB, B_h, b_bytes, cudaMemcpyHostToDevice, s_in)))
+    ok(cudaEventRecord(e_b, s_in));
+  for (int sl = 0; sl < nslab && rc == MMAEMU_OK; sl++) {
+    const size_t r0 = (size_t)sl * rows_per, rows = (size_t)(sl + 1 < nslab ? rows_per : M - (int)r0);
+    if (!ok(cudaMemcpyAsync(dA + r0 * K * ES, static_cast<const unsigned char *>(A_h) + r0 * K * ES, rows * K * ES,
+                            cudaMemcpyHostToDevice, s_in)))
+      break;
+    if (C_h && !ok(cudaMemcpyAsync(dC + r0 * N, C_h + r0 * N, rows * N * 4, cudaMemcpyHostToDevice, s_in))) break;
+    ok(cudaEventRecord(e_in(sl), s_in));
+  }
+  mmaemu::GemmParams p = row_major_params(M, N, K, dA, dB, dC, dD, dfp);
+  p.dB = buf + o_wb;
+  p.flags_b = reinterpret_cast<uint32_t *>(buf + o_fb);
+  p.batch = 1;
+  if (rc == MMAEMU_OK && ok(cudaStreamWaitEvent(t_stream, e_b, 0))) rc = launch_decode_b<MODEL, FMT>(p, 1, t_stream);
+  if (rc == MMAEMU_OK && ok(cudaEventRecord(e_bdec, t_stream))) ok(cudaStreamWaitEvent(c2, e_bdec, 0));
+  for (int sl = 0; sl < nslab && rc == MMAEMU_OK; sl++) {
+    const size_t r0 = (size_t)sl * rows_per;
+    const int rows = sl + 1 < nslab ? rows_per : M - (int)r0;
+    const cudaStream_t st = cs[sl & 1];
+    mmaemu::GemmParams q = p;
+    q.M = rows;
+    q.A = dA + r0 * K * ES;
+    q.C = dC ? dC + r0 * N : nullptr;
+    q.D = dD + r0 * N;
+    q.fp = dfp ? dfp + (r0 / 16) * (N / 16) : nullptr;
+    q.dA = buf + o_wa + (sl & 1) * up(zs.a_bytes);
+    q.flags_a = reinterpret_cast<uint32_t *>(buf + o_fa + (sl & 1) * up(zs.fa_bytes));
+    if (!ok(cudaStreamWaitEvent(st, e_in(sl), 0))) break;
+    rc = launch_decode_a_gemm<MODEL, FMT>(q, 1, st);
+    if (rc != MMAEMU_OK || !ok(cudaEventRecord(e_done(sl), st)) || !ok(cudaStreamWaitEvent(s_out, e_done(sl), 0)))
+      break;
+    if (D_h && !ok(cudaMemcpyAsync(D_h + r0 * N, dD + r0 * N, (size_t)rows * N * 4, cudaMemcpyDeviceToHost, s_out)))
+      break;
+    if (fp_h && !ok(cudaMemcpyAsync(fp_h + (r0 / 16) * (N / 16), dfp + (r0 / 16) * (N / 16),
+                                    (size_t)(rows / 16) * (N / 16) * 4, cudaMemcpyDeviceToHost, s_out)))
+      break;
+  }
+  // the buffers go back to the pool once every copy has finished
+  if (made == nev) {
+    ok(cudaEventRecord(e_out, s_out));
+    ok(cudaEventRecord(e_in(nslab - 1), s_in));
+    ok(cudaEventRecord(e_c2, c2));
+    ok(cudaStreamWaitEvent(t_stream, e_out, 0));
+    ok(cudaStreamWaitEvent(t_stream, e_in(nslab - 1), 0));
+    ok(cudaStreamWaitEvent(t_stream, e_c2, 0));
+  } else {
+    cudaStreamSynchronize(s_in);
+    cudaStreamSynchronize(s_out);
+    cudaStreamSynchronize(c2);
+  }
+  if (cudaFreeAsync(buf, t_stream) != cudaSuccess) rc = MMAEMU_ECUDA;
+  if (cudaStreamSynchronize(t_stream) != cudaSuccess) rc = MMAEMU_ECUDA;
+  for (int i = 0; i < made; i++) cudaEventDestroy(ev[i]);
   return rc;
 }
 
@@ -1382,14 +1542,6 @@ int run_gemm(int model, int fmt, mmaemu::GemmParams &p, long long batch) {
 #undef CALL_GEMM
 }
 
-mmaemu::GemmParams row_major_params(int M, int N, int K, const void *A, const void *B, const float *C, float *D,
-                                    uint32_t *fp) {
-  mmaemu::GemmParams p{};
-  p.A = A; p.B = B; p.C = C; p.D = D; p.fp = fp;
-  p.M = M; p.N = N; p.K = K;
-  p.lda = K; p.ldb = N; p.ldc = N; p.ldd = N; p.ldr = N;
-  return p;
-}
 
 template <int MODEL, int FMT>
 int launch_tiles(const void *A, const void *B, const float *C, float *D, size_t ntiles, int sms) {
@@ -1481,6 +1633,20 @@ int mmaemu_gemm_strided_batched(int model, int fmt, int trans_a, int trans_b, in
   p.sF = fingerprint_out ? stride_fp : 0;
   if (!D && !fingerprint_out) return MMAEMU_EINVAL;
   return run_gemm(model, fmt, p, batch);
+}
+
+int mmaemu_gemm_host(int model, int fmt, int M, int N, int K, const void *A, const void *B, const float *C,
+                     float *D, uint32_t *fingerprint_out) {
+  if (!valid_pair(model, fmt)) return MMAEMU_EINVAL;
+  if (!D && !fingerprint_out) return MMAEMU_EINVAL;
+  mmaemu::GemmParams p = row_major_params(M, N, K, A, B, C, D, fingerprint_out);
+  int rc = validate_gemm(p, 1);
+  if (rc != MMAEMU_OK) return rc;
+  rc = check_device();
+  if (rc != MMAEMU_OK) return rc;
+#define CALL_HOST(M_, F_) launch_gemm_host<M_, F_>(M, N, K, A, B, C, D, fingerprint_out)
+  MMAEMU_DISPATCH(model, fmt, CALL_HOST);
+#undef CALL_HOST
 }
 
 int mmaemu_xorsum(const void *D, size_t n, uint32_t *out_host) {

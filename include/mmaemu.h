@@ -161,6 +161,21 @@ int mmaemu_gemm_strided_batched(int model, int fmt, int trans_a, int trans_b, in
                                 long long ldc, long long stride_c, float *D, long long ldd,
                                 long long stride_d, uint32_t *fingerprint_out, long long stride_fp);
 
+/* mmaemu_gemm from and to HOST memory, synchronous: A, B, C (C may be NULL)
+ * and the results D and fingerprint_out (either may be NULL, not both) are
+ * host pointers; layouts and rules as mmaemu_gemm.  The call copies B and
+ * decodes it once, then streams A and C to the device in row slabs on a
+ * library-owned copy stream while earlier slabs compute on the selected
+ * stream, and copies each slab's D and fingerprints back on a second copy
+ * stream as soon as that slab is done -- the transfers overlap the
+ * arithmetic.  Page-locked host memory lets the copies run asynchronously;
+ * other host memory works too, with the copies no longer overlapped.
+ * Device memory comes from the library's workspace pool (see the GEMM
+ * implementation note).  Returns after D and the fingerprints are in host
+ * memory.  Errors: as mmaemu_gemm; MMAEMU_ECUDA also for a failed copy.  */
+int mmaemu_gemm_host(int model, int fmt, int M, int N, int K, const void *A, const void *B,
+                     const float *C, float *D, uint32_t *fingerprint_out);
+
 /* xorsum of n 32-bit words at device pointer D (the AEGIS fingerprint of a
  * whole tensor), written to *out_host.  SYNCHRONOUS: returns after the
  * result is on the host (it waits for the selected stream).  n == 0 gives 0.

@@ -43,7 +43,7 @@ def L():
 
 
 def test_header_declares_the_boundary():
-    assert declared_functions() == ["mmaemu_gemm", "mmaemu_gemm_strided_batched", "mmaemu_gemm_verify",
+    assert declared_functions() == ["mmaemu_gemm", "mmaemu_gemm_host", "mmaemu_gemm_strided_batched", "mmaemu_gemm_verify",
                                     "mmaemu_mma_emulated", "mmaemu_mma_native", "mmaemu_model_describe",
                                     "mmaemu_model_identify", "mmaemu_native_tiles",
                                     "mmaemu_probe_alignment_rounding", "mmaemu_probe_floor", "mmaemu_probe_neutral",

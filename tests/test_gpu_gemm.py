@@ -171,6 +171,29 @@ def test_workspace_reuse_and_trim(cref):
     assert np.array_equal(D, want)
 
 
+@pytest.mark.parametrize("shape", [(80, 144, 48), (1040, 400, 96), (64, 16, 16)], ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("pinned", [True, False])
+def test_gemm_from_host_memory(cref, shape, pinned):
+    """mmaemu_gemm_host: host buffers in and out, A/C/D streamed in row
+    slabs (1040 rows: five slabs of 192 and one of 80) overlapped with the
+    arithmetic -- the same bits as the device call and the oracle."""
+    import torch
+
+    import bit_exact_tensor_b200 as mmaemu
+
+    M, N, K = shape
+    A, B, C = normal_inputs(M, N, K, "fp16", seed=M + N + K)
+    host = lambda x: (torch.from_numpy(x.view(np.int32) if x.dtype == np.uint32 else x.view(np.int16)).pin_memory()
+                      if pinned else torch.from_numpy(x.view(np.int32) if x.dtype == np.uint32 else x.view(np.int16)))
+    D, fp = mmaemu.gemm_host("ampere", "fp16", host(A), host(B), host(C))
+    want = cref.gemm("ampere", "fp16", A, B, C)
+    got = D.view(torch.int32).numpy().view(np.uint32)
+    assert np.array_equal(got, want), first_mismatch(got, want)
+    assert np.array_equal(fp.numpy().view(np.uint32), cref.tile_fingerprints(want))
+    D0, _ = mmaemu.gemm_host("hopper", "fp16", host(A), host(B), None, fingerprint=False)
+    assert np.array_equal(D0.view(torch.int32).numpy().view(np.uint32), cref.gemm("hopper", "fp16", A, B, None))
+
+
 def test_null_c_in_place_and_no_fingerprint(cref):
     import bit_exact_tensor_b200 as mmaemu
 

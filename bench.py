@@ -36,7 +36,9 @@ if ROOT not in sys.path:
 
 M = N = K = 4096
 MACS_PER_STEP = M * N * K
-OPS_PER_MAC = 7  # algorithmic integer ops per emulated MAC
+# algorithmic integer ops per emulated MAC: exponent add, max, shift amount,
+# significand product, truncating shift, sign, accumulate
+OPS_PER_MAC = 7
 METRIC = "emulated MACs/s for 4096^3 FP16-Ampere GEMM; % of INT32-ALU roofline; bit-exact"
 UNIT = "MAC/s"
 # Pages' CPU simulator, same workload: 50.8 s per 4096x4096 FP16-Ampere MatMul
@@ -50,14 +52,14 @@ D2H_BYTES = M * N * 4 + (M // 16) * (N // 16) * 4
 ALGO_BYTES = H2D_BYTES + D2H_BYTES  # A, B, C read and D, fingerprints written once
 WORKLOAD = "gemm M=N=K=4096, Ampere FP16 model, fp32 C=0 and D, fused per-16x16-tile xorsum"
 # DRAM bytes per launch of the GEMM kernel (dram__bytes_read.sum + dram__bytes_write.sum)
-# from one ncu capture (profiles/gemm_ampere_fp16_4096_ncu_full.md), valid only
+# from one ncu capture (its summary is committed under profiles/), valid only
 # for the kernel sources it was taken on, identified by their hash.
 TRAFFIC_CAPTURE = {"source_sha16": "3b724c699f50b8ee", "bytes": 2_266_431_872}
 KERNEL_SOURCES = ("bit_exact_tensor_b200/csrc/mmaemu.cu", "bit_exact_tensor_b200/csrc/mmaemu_core.cuh",
                   "include/mmaemu.h")
 
 
-HBM_PEAK_GBS = 6557.4  # measured copy bandwidth on this machine's B200s (MEASURED_PEAKS.json)
+HBM_PEAK_GBS = 6557.4  # measured STREAM-style copy bandwidth of a B200, GB/s
 DEFAULT_WORKLOAD = "gemm-ampere-fp16-4096"
 PAIRS = (("ampere", "fp16"), ("ampere", "bf16"), ("hopper", "fp16"), ("hopper", "bf16"), ("hopper", "e4m3"),
          ("b200", "fp16"), ("b200", "bf16"))

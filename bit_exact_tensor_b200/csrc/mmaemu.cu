@@ -1709,7 +1709,7 @@ const char *mmaemu_strerror(int code) {
 // xorsum that allocates nothing
 //
 // For callers that cannot allocate device memory at the moment they need a
-// fingerprint -- for instance a checker that runs after the device has run out
+// fingerprint -- for instance a verification step that runs after the device has run out
 // of memory, or inside a process whose device memory is entirely reserved by
 // another allocator -- mmaemu_xorsum_noalloc does the same reduction with a
 // fixed scratch array that lives in the library image instead of a per-call

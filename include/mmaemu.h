@@ -186,7 +186,7 @@ int mmaemu_gemm_host(int model, int fmt, int M, int N, int K, const void *A, con
 int mmaemu_xorsum(const void *D, size_t n, uint32_t *out_host);
 
 /* mmaemu_xorsum for callers that cannot allocate device memory when they
- * need the fingerprint -- e.g. a checker that must still run after the device
+ * need the fingerprint -- e.g. a verification step that must still run after the device
  * has run out of memory, or a process whose device memory is wholly reserved
  * by another allocator.  It has no counterpart on the pages; it computes the
  * same value as mmaemu_xorsum.

@@ -38,8 +38,7 @@ M = N = K = 4096
 MACS_PER_STEP = M * N * K
 # algorithmic integer ops per emulated MAC in the integer formulation:
 # exponent add, max, shift amount, significand product, truncating shift,
-# sign, accumulate (the tile kernel's form, and the INT32-ALU roofline of the
-# metric)
+# sign, accumulate (the INT32-ALU roofline of the metric)
 OPS_PER_MAC = 7
 METRIC = "emulated MACs/s for 4096^3 FP16-Ampere GEMM; % of INT32-ALU roofline; bit-exact"
 UNIT = "MAC/s"
@@ -49,7 +48,7 @@ PAGES_MACS_PER_S = MACS_PER_STEP / 50.8
 # ALU issue ceiling: 148 SMs x 4 SMSPs x 32 lanes at the 1965 MHz max SM clock.
 SMS, LANES_PER_SM, MAX_SM_MHZ = 148, 128, 1965.0
 ALU_PEAK_TOPS = SMS * LANES_PER_SM * MAX_SM_MHZ * 1e6 / 1e12
-# The GEMM does each product's truncating alignment and signed accumulation
+# The kernels do each product's truncating alignment and signed accumulation
 # in one fused FP64 multiply-add (fma.rz.f64): its per-MAC work is bound by
 # the FP64 pipe, 64 lanes per SM per clock (2 cycles per warp instruction on
 # each of the 4 SMSPs) -> 148 x 64 x 1965 MHz fused multiply-adds per second.
@@ -493,21 +492,17 @@ def run_gpu(args):
         value = aggregate_value(total_ms / args.steps, world, macs)
         h2d, d2h = spec["h2d"], spec["d2h"]
         int_ops = OPS_PER_MAC * macs / (kern_ms / 1e3) / 1e12
-        if spec["kind"] == "gemm":
-            # one fused FP64 multiply-add per emulated MAC
-            achieved = macs / (kern_ms / 1e3) / 1e12
-            roof = {"bound": "alu", "achieved": achieved, "peak": FP64_PEAK_TFMAS, "unit": "T FMA/s",
-                    "frac": achieved / FP64_PEAK_TFMAS,
-                    "kernel": f"gemm_kernel<{spec['model']},{spec['fmt']}> with its decode pass (one call, timed whole)",
-                    "fma_per_mac": 1, "peak_basis": "148 SM x 64 FP64 lanes x 1965 MHz (derived)",
-                    # the metric's INT32-ALU roofline: the integer formulation's
-                    # 7 ops per MAC against the INT32 issue ceiling
-                    "int32_alu_frac": int_ops / ALU_PEAK_TOPS, "int32_alu_peak_tops": ALU_PEAK_TOPS,
-                    "ops_per_mac_integer_form": OPS_PER_MAC}
-        else:
-            roof = {"bound": "alu", "achieved": int_ops, "peak": ALU_PEAK_TOPS, "unit": "Tops/s",
-                    "frac": int_ops / ALU_PEAK_TOPS, "kernel": f"tiles_kernel<{spec['model']},{spec['fmt']}>",
-                    "ops_per_mac": OPS_PER_MAC, "peak_basis": "148 SM x 128 lanes x 1965 MHz issue ceiling (derived)"}
+        # one fused FP64 multiply-add per emulated MAC
+        achieved = macs / (kern_ms / 1e3) / 1e12
+        kernel = (f"gemm_kernel<{spec['model']},{spec['fmt']}> with its decode pass (one call, timed whole)"
+                  if spec["kind"] == "gemm" else f"tiles_kernel<{spec['model']},{spec['fmt']}>")
+        roof = {"bound": "alu", "achieved": achieved, "peak": FP64_PEAK_TFMAS, "unit": "T FMA/s",
+                "frac": achieved / FP64_PEAK_TFMAS, "kernel": kernel,
+                "fma_per_mac": 1, "peak_basis": "148 SM x 64 FP64 lanes x 1965 MHz (derived)",
+                # the metric's INT32-ALU roofline: the integer formulation's
+                # 7 ops per MAC against the INT32 issue ceiling
+                "int32_alu_frac": int_ops / ALU_PEAK_TOPS, "int32_alu_peak_tops": ALU_PEAK_TOPS,
+                "ops_per_mac_integer_form": OPS_PER_MAC}
         roof.update({"traffic": measured_traffic() if args.workload == DEFAULT_WORKLOAD else None,
                      "traffic_unit": "bytes per launch", "algorithmic_bytes": h2d + d2h})
         if spec["kind"] == "tiles":  # mixed bound: also report HBM against the measured copy bandwidth

@@ -8,13 +8,11 @@
 //   xorsum_kernel -- XOR of a buffer of 32-bit words.
 // The arithmetic itself is in mmaemu_core.cuh; see the model citations there.
 // Tensor cores are deliberately not used: B200's own MMA arithmetic is not the
-// arithmetic being emulated.  Everything is exact: the tile kernel works in
-// integers, balanced between the ALU pipe (shifts, logic, min, add) and the
-// IMAD pipe (products and sign-carrying accumulation); the GEMM keeps the
-// exponent-max pass in packed integers and does each product's truncating
-// alignment and signed accumulation in one fused FP64 multiply-add with
-// round-toward-zero, on an integer held in a double's mantissa (see
-// group_products for double panels).
+// arithmetic being emulated.  Everything is exact: both kernels keep the
+// exponent-max pass, the carried terms and the write-back in integer (or
+// exact float) steps, and do each product's truncating alignment and signed
+// accumulation in one fused FP64 multiply-add with round-toward-zero, on an
+// integer held in a double's mantissa (see group_products).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -29,28 +27,12 @@ namespace mmaemu {
 // ---------------------------------------------------------------------------
 // decoded operand panels in shared memory, [k][row] for A and [k][col] for B
 // ---------------------------------------------------------------------------
-// Product signs are applied by an IMAD with sigma_a * sigma_b (+-1): on B200
-// that keeps the sign work on the IMAD pipe, which the shifts and adds of the
-// alignment leave half idle.  (Folding sigma_a into A's significand with its
-// sign mask as the IMAD addend saves one IMAD per product but needs a
-// popcount correction per group; measured slower.)
+// Operand panels of one 16-deep K chunk: the operands as exact doubles for
+// the fused truncate-and-add step of group_products below, the packed
+// negated exponents of the max pass, and the chunk's sign bits per row of A
+// and per column of B.
 template <int BM, int BN>
 struct __align__(16) Panel {
-  uint32_t aM[16][BM];   // ma << (F - 2p): one IMAD with mb gives the term magnitude
-  int32_t aN[16][BM];    // -ea (ZSENT / NINF / NNAN markers)
-  int32_t aP[16][BM];    // sign as +-1
-  uint32_t aN2[16][BM];  // (-ea, -ea) packed pair, for the packed max pass
-  uint32_t bM[16][BN];
-  int32_t bN[16][BN];
-  int32_t bP[16][BN];    // sign as +-1
-  int16_t bN2[16][BN];   // -eb as 16-bit: adjacent columns read as one pair
-};
-
-// GEMM panels: the operands as exact doubles for the fused truncate-and-add
-// step of group_products below, the packed negated exponents of the max
-// pass, and the chunk's sign bits per row of A and per column of B.
-template <int BM, int BN>
-struct __align__(16) DPanel {
   double aV[16][BM];     // A value; zero, Inf and NaN as +-2^-500
   uint32_t aN2[16][BM];  // (-ea, -ea) packed (ZSENT / NINF / NNAN markers)
   uint16_t aS[BM];       // bit k: sign of A[m][k]
@@ -59,7 +41,8 @@ struct __align__(16) DPanel {
   uint16_t bS[BN];       // bit k: sign of B[k][n]
 };
 
-// Slot of column n (0..BN-1) in a row of bV.  A thread reads its 8
+// Slot of column n (0..BN-1) in a row of bV in the GEMM's panels (the tile
+// kernel's panels keep natural order).  A GEMM thread reads its 8
 // consecutive columns as 4 pairs, and the 4 threads of a quarter warp read
 // 4 column groups 64 bytes apart, which would put groups 0 and 2 (and 1 and
 // 3) on the same banks; storing pair q of group g at pair q ^ (g & 2) gives
@@ -70,42 +53,24 @@ __host__ __device__ constexpr int bv_slot(int n) {
 
 // Per-element reads used off the main path (zero-sign rule, Inf/NaN).
 template <int BM, int BN>
-__device__ __forceinline__ int32_t n_a(const Panel<BM, BN> &P, int k, int m) { return P.aN[k][m]; }
+__device__ __forceinline__ int32_t n_a(const Panel<BM, BN> &P, int k, int m) { return lo16(P.aN2[k][m]); }
 template <int BM, int BN>
-__device__ __forceinline__ int32_t n_b(const Panel<BM, BN> &P, int k, int n) { return P.bN[k][n]; }
+__device__ __forceinline__ int32_t n_b(const Panel<BM, BN> &P, int k, int n) { return P.bN2[k][n]; }
 template <int BM, int BN>
-__device__ __forceinline__ bool neg_a(const Panel<BM, BN> &P, int k, int m) { return P.aP[k][m] < 0; }
+__device__ __forceinline__ bool neg_a(const Panel<BM, BN> &P, int k, int m) { return (P.aS[m] >> k) & 1u; }
 template <int BM, int BN>
-__device__ __forceinline__ bool neg_b(const Panel<BM, BN> &P, int k, int n) { return P.bP[k][n] < 0; }
-template <int BM, int BN>
-__device__ __forceinline__ int32_t n_a(const DPanel<BM, BN> &P, int k, int m) { return lo16(P.aN2[k][m]); }
-template <int BM, int BN>
-__device__ __forceinline__ int32_t n_b(const DPanel<BM, BN> &P, int k, int n) { return P.bN2[k][n]; }
-template <int BM, int BN>
-__device__ __forceinline__ bool neg_a(const DPanel<BM, BN> &P, int k, int m) { return (P.aS[m] >> k) & 1u; }
-template <int BM, int BN>
-__device__ __forceinline__ bool neg_b(const DPanel<BM, BN> &P, int k, int n) { return (P.bS[n] >> k) & 1u; }
+__device__ __forceinline__ bool neg_b(const Panel<BM, BN> &P, int k, int n) { return (P.bS[n] >> k) & 1u; }
 
-// Unroll of the k loops per model and format, for the integer panels (tile
-// kernel) and the double panels (GEMM).  Measured: integer panels 4 for
-// Ampere FP16 and the B200 model, else 2; double panels 4 for Ampere FP16,
-// 1 for the B200 model (its 64-bit carry keeps more registers live), else 2.
+// Unroll of the k loops per model and format (measured on the GEMM: 4 for
+// Ampere FP16, 1 for the B200 model, whose 64-bit carry keeps more registers
+// live, else 2).
 #ifndef MMAEMU_KUNROLL
 template <int MODEL, int FMT>
-constexpr int kUnroll = (MODEL == MODEL_AMPERE && FMT == FMT_FP16) || MODEL == MODEL_B200 ? 4 : 2;
-template <int MODEL, int FMT>
-constexpr int kUnrollD = MODEL == MODEL_AMPERE && FMT == FMT_FP16 ? 4 : MODEL == MODEL_B200 ? 1 : 2;
+constexpr int kUnroll = MODEL == MODEL_AMPERE && FMT == FMT_FP16 ? 4 : MODEL == MODEL_B200 ? 1 : 2;
 #else
 template <int MODEL, int FMT>
 constexpr int kUnroll = MMAEMU_KUNROLL;
-template <int MODEL, int FMT>
-constexpr int kUnrollD = MMAEMU_KUNROLL;
 #endif
-
-template <class PanelT> struct IsDPanel { static constexpr bool value = false; };
-template <int BM, int BN> struct IsDPanel<DPanel<BM, BN>> { static constexpr bool value = true; };
-template <int MODEL, int FMT, class PanelT>
-constexpr int kUnrollFor = IsDPanel<PanelT>::value ? kUnrollD<MODEL, FMT> : kUnroll<MODEL, FMT>;
 
 template <int R, typename T>
 __device__ __forceinline__ void lds_vec(const T *p, T (&v)[R]) {
@@ -158,32 +123,6 @@ __device__ __forceinline__ void group_max(const PanelT &P, int rl, int cl, const
     }
 }
 
-// Pass 2 of a group: add every product's aligned (truncated) magnitude, with
-// its sign, to S (which already holds the carried term's contribution).
-template <int F, int K0, int KN, int R, int CC, int UNR, int BM, int BN>
-__device__ __forceinline__ void group_products(const Panel<BM, BN> &P, int rl, int cl, const int32_t (&nmin)[R][CC],
-                                               int32_t (&S)[R][CC]) {
-#pragma unroll UNR
-  for (int k = K0; k < K0 + KN; k++) {
-    uint32_t am[R], bm[CC];
-    int32_t an[R], ap[R], bn[CC], bp[CC];
-    lds_vec<R>(&P.aM[k][rl], am);
-    lds_vec<R>(&P.aN[k][rl], an);
-    lds_vec<R>(&P.aP[k][rl], ap);
-    lds_vec<CC>(&P.bM[k][cl], bm);
-    lds_vec<CC>(&P.bN[k][cl], bn);
-    lds_vec<CC>(&P.bP[k][cl], bp);
-    // column-outer order: measured faster (operand reuse across rows)
-#pragma unroll
-    for (int c = 0; c < CC; c++)
-#pragma unroll
-      for (int r = 0; r < R; r++) {
-        const uint32_t T = shr_u32(am[r] * bm[c], (uint32_t)(an[r] + bn[c] - nmin[r][c]));
-        S[r][c] += (int32_t)T * (ap[r] * bp[c]);
-      }
-  }
-}
-
 __device__ __forceinline__ double fma_rz(double a, double b, double c) {
   double d;
   asm("fma.rz.f64 %0, %1, %2, %3;" : "=d"(d) : "d"(a), "d"(b), "d"(c));
@@ -201,7 +140,9 @@ __device__ __forceinline__ void lds_dvec(const double *p, double (&v)[R]) {
   }
 }
 
-// The same pass on double panels, one fused multiply-add per product.
+// Pass 2 of a group: add every product's aligned (truncated) magnitude, with
+// its sign, to S (which holds the carried term's contribution), with one
+// fused multiply-add per product.
 // Per output, acc holds (2^52 + 2^51 + L) u on the group's grid u =
 // 2^(e_max - F), with L = S mod 2^32 in its low mantissa bits; every double
 // in [2^52 u, 2^53 u) is a multiple of u, so fma.rz(a, b', acc) -- one
@@ -223,7 +164,7 @@ __device__ __forceinline__ void lds_dvec(const double *p, double (&v)[R]) {
 // term (or is overwritten as Inf/NaN), and every product of a zero stand-in
 // (below 2^-371) truncates to zero on it.
 template <int F, int K0, int KN, int R, int CC, int UNR, int BM, int BN>
-__device__ __forceinline__ void group_products(const DPanel<BM, BN> &P, int rl, int cl,
+__device__ __forceinline__ void group_products(const Panel<BM, BN> &P, int rl, int cl,
                                                const int32_t (&nmin)[R][CC], int32_t (&S)[R][CC]) {
   double acc[R][CC];
   constexpr uint32_t HI0 = ((uint32_t)(1075 - F) << 20) | 0x80000u;
@@ -232,17 +173,23 @@ __device__ __forceinline__ void group_products(const DPanel<BM, BN> &P, int rl, 
 #pragma unroll
     for (int c = 0; c < CC; c++)
       acc[r][c] = __hiloint2double((int)(HI0 - ((uint32_t)nmin[r][c] << 20)), S[r][c]);
-  static_assert(CC == 8, "bV holds 8-column groups with their pairs swizzled");
-  const int sw = (cl >> 3) & 2;  // see bv_slot
+  // 8-column groups (GEMM) are stored with their pairs swizzled (bv_slot);
+  // 4-column groups (tile kernel) in natural order, which is conflict-free
+  static_assert(CC == 8 || CC == 4, "column groups of 8 or 4");
+  const int sw = (cl >> 3) & 2;
 #pragma unroll UNR
   for (int k = K0; k < K0 + KN; k++) {
     double a[R], b[CC];
     lds_dvec<R>(&P.aV[k][rl], a);
+    if constexpr (CC == 8) {
 #pragma unroll
-    for (int q = 0; q < 4; q++) {
-      const double2 t = *reinterpret_cast<const double2 *>(&P.bV[k][cl + 2 * (q ^ sw)]);
-      b[2 * q] = t.x;
-      b[2 * q + 1] = t.y;
+      for (int q = 0; q < 4; q++) {
+        const double2 t = *reinterpret_cast<const double2 *>(&P.bV[k][cl + 2 * (q ^ sw)]);
+        b[2 * q] = t.x;
+        b[2 * q + 1] = t.y;
+      }
+    } else {
+      lds_dvec<CC>(&P.bV[k][cl], b);
     }
 #pragma unroll
     for (int c = 0; c < CC; c++)
@@ -359,7 +306,7 @@ template <int MODEL, int FMT, int R, int CC, class PanelT>
 __device__ __forceinline__ void mma_chunk(const PanelT &P, int rl, int cl, uint32_t (&Np)[R][CC / 2],
                                           int32_t (&X)[R][CC], uint32_t &dneg0, bool panel_special) {
   constexpr int F = ModelT<MODEL>::F;
-  constexpr int UNR = kUnrollFor<MODEL, FMT, PanelT>;
+  constexpr int UNR = kUnroll<MODEL, FMT>;
   static_assert(R * CC <= 32 && CC % 2 == 0, "per-output masks hold 32 outputs");
   // with 24 or more fraction bits the grid would see state bits below the
   // fp32 value's 24: keep bits 0..6 clear
@@ -578,7 +525,7 @@ __device__ __forceinline__ void mma_chunk_fast(const PanelT &P, int rl, int cl, 
   int32_t S[R][CC], nmin[R][CC];
   constexpr int KN1 = MODEL == MODEL_AMPERE ? 8 : 16;
   constexpr bool WIDE = kWideSum<MODEL>;
-  constexpr int UNR = kUnrollFor<MODEL, FMT, PanelT>;
+  constexpr int UNR = kUnroll<MODEL, FMT>;
   // first (or only) group: carried D plus products (the carried term is
   // added in the write-back when the sum may need 33 bits)
   group_max<FMT, 0, KN1, R, CC, UNR>(P, rl, cl, Np, nmin);
@@ -860,36 +807,46 @@ __device__ __forceinline__ Raw8<FMT> load_col8(const void *base, size_t elem_off
   return r;
 }
 
-// Decode 8 k-consecutive elements of A row m (k = 8h .. 8h+7) into the panel.
+// Exact value of a decoded element as a double, m 2^(e - p) with its sign;
+// zero, Inf and NaN become +-2^-500 (the special-value path reads their
+// markers instead).
+template <int FMT>
+__device__ __forceinline__ double dec_value(const Dec &d) {
+  constexpr int P = FmtT<FMT>::P;
+  const double scale = __hiloint2double((1023 - d.n - P) << 20, 0);  // 2^(e - p), normal for every format
+  const double v = d.m ? (double)d.m * scale : 0x1p-500;
+  return d.s ? -v : v;
+}
+
+// Decode 8 k-consecutive elements of A row m (k = 8h .. 8h+7) into a tile
+// kernel's panel (4-column groups, natural order), or of B column n.
 template <int MODEL, int FMT, int BM, int BN>
 __device__ __forceinline__ uint32_t store_a8(Panel<BM, BN> &P, int m, int h, const Raw8<FMT> &raw) {
-  constexpr int SH = ModelT<MODEL>::F - 2 * FmtT<FMT>::P;
-  uint32_t special = 0;
+  uint32_t special = 0, signs = 0;
 #pragma unroll
   for (int i = 0; i < 8; i++) {
     const Dec d = decode<FMT>(raw.get(i));
-    P.aM[8 * h + i][m] = d.m << SH;
-    P.aN[8 * h + i][m] = d.n;
-    P.aP[8 * h + i][m] = (int32_t)(d.s | 1u);
+    P.aV[8 * h + i][m] = dec_value<FMT>(d);
     P.aN2[8 * h + i][m] = pack16(d.n, d.n);
+    signs |= (d.s & 1u) << i;
     special |= d.special;
   }
+  reinterpret_cast<uint8_t *>(&P.aS[m])[h] = (uint8_t)signs;
   return special;
 }
 
-// Decode 8 k-consecutive elements of B column n (k = 8h .. 8h+7).
 template <int FMT, int BM, int BN>
 __device__ __forceinline__ uint32_t store_b8(Panel<BM, BN> &P, int n, int h, const Raw8<FMT> &raw) {
-  uint32_t special = 0;
+  uint32_t special = 0, signs = 0;
 #pragma unroll
   for (int i = 0; i < 8; i++) {
     const Dec d = decode<FMT>(raw.get(i));
-    P.bM[8 * h + i][n] = d.m;
-    P.bN[8 * h + i][n] = d.n;
-    P.bP[8 * h + i][n] = (int32_t)(d.s | 1u);
+    P.bV[8 * h + i][n] = dec_value<FMT>(d) * (1.0 + 0x1p-40);  // exact
     P.bN2[8 * h + i][n] = (int16_t)d.n;
+    signs |= (d.s & 1u) << i;
     special |= d.special;
   }
+  reinterpret_cast<uint8_t *>(&P.bS[n])[h] = (uint8_t)signs;
   return special;
 }
 
@@ -901,7 +858,7 @@ __device__ __forceinline__ uint32_t store_b8(Panel<BM, BN> &P, int n, int h, con
 #define MMAEMU_GMINB 2
 #endif
 constexpr int GBM = 64, GBN = 128, GTHREADS = 256, GR = 4, GCC = 8;
-using GPanel = DPanel<GBM, GBN>;
+using GPanel = Panel<GBM, GBN>;
 
 // Everything a GEMM launch needs.  Element (m, k) of op(A) sits at
 // A[m * lda + k] (ta == 0) or A[k * lda + m] (ta == 1); element (k, n) of
@@ -935,17 +892,6 @@ static_assert(ABLOB == 12416 && BBLOB == 20736, "panel layout");
 static_assert(offsetof(GPanel, aN2) == 8192 && offsetof(GPanel, aS) == 12288 &&
                   offsetof(GPanel, bN2) - ABLOB == 16384 && offsetof(GPanel, bS) - ABLOB == 20480,
               "blob field offsets");
-
-// Exact value of a decoded element as a double, m 2^(e - p) with its sign;
-// zero, Inf and NaN become +-2^-500 (the special-value path reads their
-// markers instead).
-template <int FMT>
-__device__ __forceinline__ double dec_value(const Dec &d) {
-  constexpr int P = FmtT<FMT>::P;
-  const double scale = __hiloint2double((1023 - d.n - P) << 20, 0);  // 2^(e - p), normal for every format
-  const double v = d.m ? (double)d.m * scale : 0x1p-500;
-  return d.s ? -v : v;
-}
 
 // Decode pass, A side: one thread per 8 k-consecutive elements (row m,
 // chunk j, half h) into the blob of (batch entry, m / 64, j).

@@ -854,10 +854,18 @@ __device__ __forceinline__ uint32_t store_b8(Panel<BM, BN> &P, int n, int h, con
 // GEMM
 // ---------------------------------------------------------------------------
 // Tuning knobs (compile-time): resident blocks per SM and the unroll of the k loops.
-#ifndef MMAEMU_GMINB
-#define MMAEMU_GMINB 2
+// A block computes GBM x GBN outputs with one warp per 32 x 32 and a 4 x 8
+// block of outputs per thread.  Measured: 64 x 64 blocks of 128 threads, 4
+// per SM, are 3-5% faster than 64 x 128 blocks of 256 threads, 2 per SM (the
+// same registers and warps per SM, but half as many warps wait at each
+// block's per-chunk barrier).
+#ifndef MMAEMU_GBN
+#define MMAEMU_GBN 64
 #endif
-constexpr int GBM = 64, GBN = 128, GTHREADS = 256, GR = 4, GCC = 8;
+#ifndef MMAEMU_GMINB
+#define MMAEMU_GMINB (256 / MMAEMU_GBN)
+#endif
+constexpr int GBM = 64, GBN = MMAEMU_GBN, GWN = GBN / 32, GTHREADS = 32 * 2 * GWN, GR = 4, GCC = 8;
 using GPanel = Panel<GBM, GBN>;
 
 // Everything a GEMM launch needs.  Element (m, k) of op(A) sits at
@@ -888,10 +896,11 @@ struct GemmParams {
 // Decoded panel blobs: the A part (aV, aN2, aS) and the B part (bV, bN2,
 // bS) of a GPanel, stored contiguously in that order.
 constexpr size_t ABLOB = offsetof(GPanel, bV), BBLOB = sizeof(GPanel) - offsetof(GPanel, bV);
-static_assert(ABLOB == 12416 && BBLOB == 20736, "panel layout");
-static_assert(offsetof(GPanel, aN2) == 8192 && offsetof(GPanel, aS) == 12288 &&
-                  offsetof(GPanel, bN2) - ABLOB == 16384 && offsetof(GPanel, bS) - ABLOB == 20480,
-              "blob field offsets");
+constexpr size_t OFF_AN2 = offsetof(GPanel, aN2), OFF_AS = offsetof(GPanel, aS);
+constexpr size_t OFF_BN2 = offsetof(GPanel, bN2) - ABLOB, OFF_BS = offsetof(GPanel, bS) - ABLOB;
+static_assert(ABLOB == 16 * GBM * 8 + 16 * GBM * 4 + GBM * 2 && BBLOB == 16 * GBN * 8 + 16 * GBN * 2 + GBN * 2 &&
+                  ABLOB % 16 == 0 && BBLOB % 16 == 0,
+              "panel layout");
 
 // Decode pass, A side: one thread per 8 k-consecutive elements (row m,
 // chunk j, half h) into the blob of (batch entry, m / 64, j).
@@ -915,11 +924,11 @@ __global__ void __launch_bounds__(256) decode_a_kernel(const GemmParams p) {
     const Dec d = decode<FMT>(raw.get(i));
     const size_t kk = (size_t)(8 * h + i);
     *reinterpret_cast<double *>(blob + (kk * GBM + ml) * 8) = dec_value<FMT>(d);
-    *reinterpret_cast<uint32_t *>(blob + 8192 + (kk * GBM + ml) * 4) = pack16(d.n, d.n);
+    *reinterpret_cast<uint32_t *>(blob + OFF_AN2 + (kk * GBM + ml) * 4) = pack16(d.n, d.n);
     signs |= (d.s & 1u) << i;
     special |= d.special;
   }
-  blob[12288 + 2 * ml + h] = (unsigned char)signs;
+  blob[OFF_AS + 2 * ml + h] = (unsigned char)signs;
   if (special) atomicOr(&p.flags_a[(bz * nrb + rb) * nch + j], 1u);
 }
 
@@ -944,11 +953,11 @@ __global__ void __launch_bounds__(256) decode_b_kernel(const GemmParams p) {
     const Dec d = decode<FMT>(raw.get(i));
     const size_t kk = (size_t)(8 * h + i);
     *reinterpret_cast<double *>(blob + (kk * GBN + bv_slot(nl)) * 8) = dec_value<FMT>(d) * (1.0 + 0x1p-40);  // exact
-    *reinterpret_cast<int16_t *>(blob + 16384 + (kk * GBN + nl) * 2) = (int16_t)d.n;
+    *reinterpret_cast<int16_t *>(blob + OFF_BN2 + (kk * GBN + nl) * 2) = (int16_t)d.n;
     signs |= (d.s & 1u) << i;
     special |= d.special;
   }
-  blob[20480 + 2 * nl + h] = (unsigned char)signs;
+  blob[OFF_BS + 2 * nl + h] = (unsigned char)signs;
   if (special) atomicOr(&p.flags_b[(bz * ncb + cb) * nch + j], 1u);
 }
 
@@ -985,12 +994,12 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const Gemm
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row0 = rb * GBM, col0 = cb * GBN;
   // this thread's 4 x 8 outputs
-  const int rl = (warp >> 2) * 32 + (lane >> 2) * GR;
-  const int cl = (warp & 3) * 32 + (lane & 3) * GCC;
+  const int rl = (warp / GWN) * 32 + (lane >> 2) * GR;
+  const int cl = (warp % GWN) * 32 + (lane & 3) * GCC;
   const bool out_valid = (row0 + rl < M) && (col0 + cl < N);
 
-  // Per chunk, the block copies its decoded A and B blobs (12,416 + 20,736
-  // bytes) into the panel with 16-byte asynchronous copies: 776 + 1,296.
+  // Per chunk, the block copies its decoded A and B blobs (12,416 + 10,368
+  // bytes for 64 x 64 blocks) into the panel with 16-byte asynchronous copies.
   const int nchunks = K / 16;
   const unsigned char *blob_a = p.dA + (bz * nrb + rb) * (size_t)nchunks * ABLOB;
   const unsigned char *blob_b = p.dB + (bz * ncb + cb) * (size_t)nchunks * BBLOB;

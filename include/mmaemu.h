@@ -88,7 +88,7 @@ int mmaemu_tiles(int model, int fmt, const void *A, const void *B, const float *
  * A and B once into panel form, then the MMA kernel copies those panels
  * instead of decoding per output block.  The decoded operands live in a
  * stream-ordered workspace of
- *   batch * K/16 * (ceil(M/64) * 12416 + ceil(N/128) * 20736 + small)
+ *   batch * K/16 * (ceil(M/64) * 12416 + ceil(N/64) * 10368 + small)
  * bytes (about 375 MB for M = N = K = 4096) taken from a memory pool owned
  * by the library.  Freed workspace stays in that pool for the next call;
  * mmaemu_trim_workspace hands it back to the device.  A failed workspace

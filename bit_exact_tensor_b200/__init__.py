@@ -16,13 +16,22 @@ import os
 import threading
 
 __all__ = ["MODELS", "FORMATS", "MmaEmuError", "lib", "tiles", "gemm", "gemm_verify", "gemm_batched", "xorsum",
-           "xorsum_noalloc", "gemm_host", "set_stream", "trim_workspace", "NO_MISMATCH"]
+           "xorsum_noalloc", "gemm_host", "set_stream", "trim_workspace", "set_workspace_cache", "workspace_reserved",
+           "device_status", "selftest_wait_timeout", "bounds_checking", "NO_MISMATCH"]
 
 MODELS = {"ampere": 0, "hopper": 1, "b200": 2, "lovelace": 0}
 FORMATS = {"fp16": 0, "bf16": 1, "e4m3": 2}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmmaemu.so")
+# MMAEMU_LIB=check selects the bounds-checking build (libmmaemu_check.so):
+# every kernel index is checked against its buffer and a violation is
+# recorded in the device status word (see device_status) instead of being
+# made.  It is slower and meant for tests.  MMAEMU_LIB=<path to a .so>
+# loads another build of the same sources (for instance one compiled with
+# other tuning constants).
+_SEL = os.environ.get("MMAEMU_LIB", "")
+LIB_PATH = (os.path.join(_HERE, "libmmaemu_check.so") if _SEL == "check"
+            else _SEL if _SEL.endswith(".so") else os.path.join(_HERE, "libmmaemu.so"))
 _lock = threading.Lock()
 _lib = None
 
@@ -60,6 +69,18 @@ def lib() -> ctypes.CDLL:
             L.mmaemu_xorsum.restype = i32
             L.mmaemu_strerror.argtypes = [i32]
             L.mmaemu_strerror.restype = ctypes.c_char_p
+            L.mmaemu_set_workspace_cache.argtypes = [i32]
+            L.mmaemu_set_workspace_cache.restype = i32
+            L.mmaemu_workspace_reserved.argtypes = [ctypes.POINTER(sz)]
+            L.mmaemu_workspace_reserved.restype = i32
+            L.mmaemu_trim_workspace.argtypes = []
+            L.mmaemu_trim_workspace.restype = i32
+            L.mmaemu_device_status.argtypes = [i32, ctypes.POINTER(ctypes.c_uint32)]
+            L.mmaemu_device_status.restype = i32
+            L.mmaemu_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.POINTER(i32)]
+            L.mmaemu_selftest_wait_timeout.restype = i32
+            L.mmaemu_bounds_checking.argtypes = []
+            L.mmaemu_bounds_checking.restype = i32
             _lib = L
         return _lib
 
@@ -83,6 +104,37 @@ def set_stream(stream=None):
         stream = torch.cuda.current_stream()
     handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
     _check(lib().mmaemu_set_stream(ctypes.c_void_p(handle)), "mmaemu_set_stream")
+
+
+def _device_of(*tensors):
+    """The one CUDA device all given tensors live on (None entries are
+    skipped); raises before any launch if they differ.  Calls run with that
+    device current and on its current stream, so a tensor on another GPU
+    than the current one is never handed to a kernel on the wrong device."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"operands must all be on one CUDA device, got {sorted(str(d) for d in devs)}")
+    (dev,) = devs
+    if dev.type != "cuda":
+        raise TypeError("operands must be CUDA tensors")
+    return dev
+
+
+class _on_device:
+    """Context: make ``dev`` current and select its current stream."""
+
+    def __init__(self, dev):
+        self.dev = dev
+
+    def __enter__(self):
+        torch = _torch()
+        self.ctx = torch.cuda.device(self.dev)
+        self.ctx.__enter__()
+        set_stream(torch.cuda.current_stream(self.dev))
+        return self
+
+    def __exit__(self, *exc):
+        return self.ctx.__exit__(*exc)
 
 
 _IN_DTYPES = None
@@ -141,9 +193,9 @@ def tiles(model: str, fmt: str, A, B, C=None, out=None):
         out = torch.empty((nt, 16, 16), dtype=torch.float32, device=A.device)
     else:
         _check_f32(out, "out")
-    set_stream()
-    _check(lib().mmaemu_tiles(mi, fi, A.data_ptr(), B.data_ptr(), C.data_ptr() if C is not None else None,
-                              out.data_ptr(), nt), "mmaemu_tiles")
+    with _on_device(_device_of(A, B, C, out)):
+        _check(lib().mmaemu_tiles(mi, fi, A.data_ptr(), B.data_ptr(), C.data_ptr() if C is not None else None,
+                                  out.data_ptr(), nt), "mmaemu_tiles")
     return out
 
 
@@ -181,10 +233,13 @@ def gemm(model: str, fmt: str, A, B, C=None, out=None, fingerprint: bool = True,
     if fingerprint:
         fp = fp_out if fp_out is not None else torch.empty(((M // 16) * (N // 16),), dtype=torch.int32,
                                                            device=A.device)
-    set_stream()
-    _check(lib().mmaemu_gemm(mi, fi, M, N, K, A.data_ptr(), B.data_ptr(),
-                             C.data_ptr() if C is not None else None, out.data_ptr() if out is not None else None,
-                             fp.data_ptr() if fp is not None else None), "mmaemu_gemm")
+    if fp is not None and (not fp.is_cuda or fp.numel() != (M // 16) * (N // 16) or fp.element_size() != 4
+                           or not fp.is_contiguous()):
+        raise ValueError("fp_out must be a contiguous CUDA tensor of (M/16)*(N/16) 32-bit words")
+    with _on_device(_device_of(A, B, C, out, fp)):
+        _check(lib().mmaemu_gemm(mi, fi, M, N, K, A.data_ptr(), B.data_ptr(),
+                                 C.data_ptr() if C is not None else None, out.data_ptr() if out is not None else None,
+                                 fp.data_ptr() if fp is not None else None), "mmaemu_gemm")
     return out, fp
 
 
@@ -207,11 +262,11 @@ def gemm_verify(model: str, fmt: str, A, B, C, D_claimed, fingerprint: bool = Fa
     if mism.dtype != torch.int64 or mism.numel() != 2 or not mism.is_cuda:
         raise TypeError("mismatch_out must be a CUDA int64 tensor of 2 elements")
     fp = torch.empty(((M // 16) * (N // 16),), dtype=torch.int32, device=A.device) if fingerprint else None
-    set_stream()
-    _check(lib().mmaemu_gemm_verify(mi, fi, M, N, K, A.data_ptr(), B.data_ptr(),
-                                    C.data_ptr() if C is not None else None, D_claimed.data_ptr(),
-                                    fp.data_ptr() if fp is not None else None, mism.data_ptr()),
-           "mmaemu_gemm_verify")
+    with _on_device(_device_of(A, B, C, D_claimed, fp, mism)):
+        _check(lib().mmaemu_gemm_verify(mi, fi, M, N, K, A.data_ptr(), B.data_ptr(),
+                                        C.data_ptr() if C is not None else None, D_claimed.data_ptr(),
+                                        fp.data_ptr() if fp is not None else None, mism.data_ptr()),
+               "mmaemu_gemm_verify")
     return mism, fp
 
 
@@ -275,13 +330,13 @@ def gemm_batched(model: str, fmt: str, A, B, C=None, out=None, fingerprint: bool
         raise ValueError("out entries of a batch must not overlap")
     tiles_per = (M // 16) * (N // 16)
     fp = torch.empty((batch, tiles_per), dtype=torch.int32, device=A.device) if fingerprint else None
-    set_stream()
-    _check(lib().mmaemu_gemm_strided_batched(
-        mi, fi, ta, tb, M, N, K, batch,
-        A.data_ptr(), lda, sa, B.data_ptr(), ldb, sb,
-        C.data_ptr() if C is not None else None, ldc, sc,
-        out.data_ptr() if out is not None else None, ldd, sd,
-        fp.data_ptr() if fp is not None else None, tiles_per), "mmaemu_gemm_strided_batched")
+    with _on_device(_device_of(A, B, C, out, fp)):
+        _check(lib().mmaemu_gemm_strided_batched(
+            mi, fi, ta, tb, M, N, K, batch,
+            A.data_ptr(), lda, sa, B.data_ptr(), ldb, sb,
+            C.data_ptr() if C is not None else None, ldc, sc,
+            out.data_ptr() if out is not None else None, ldd, sd,
+            fp.data_ptr() if fp is not None else None, tiles_per), "mmaemu_gemm_strided_batched")
     return out, fp
 
 
@@ -294,8 +349,8 @@ def xorsum(t) -> int:
     if nbytes % 4:
         raise ValueError("tensor size must be a whole number of 32-bit words")
     res = ctypes.c_uint32(0)
-    set_stream()
-    _check(lib().mmaemu_xorsum(t.data_ptr(), nbytes // 4, ctypes.byref(res)), "mmaemu_xorsum")
+    with _on_device(_device_of(t)):
+        _check(lib().mmaemu_xorsum(t.data_ptr(), nbytes // 4, ctypes.byref(res)), "mmaemu_xorsum")
     return int(res.value)
 
 
@@ -323,7 +378,7 @@ def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bo
     D_host = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
     fp_host = torch.empty(((M // 16) * (N // 16),), dtype=torch.int32, pin_memory=True) if fingerprint else None
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
-        set_stream()
+        set_stream(torch.cuda.current_stream())
         fn = lib().mmaemu_gemm_host
         fn.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 5
         fn.restype = ctypes.c_int
@@ -354,8 +409,8 @@ def xorsum_noalloc(t) -> int:
     fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32)]
     fn.restype = ctypes.c_int
     res = ctypes.c_uint32(0)
-    set_stream()
-    _check(fn(t.data_ptr(), nbytes // 4, ctypes.byref(res)), "mmaemu_xorsum_noalloc")
+    with _on_device(_device_of(t)):
+        _check(fn(t.data_ptr(), nbytes // 4, ctypes.byref(res)), "mmaemu_xorsum_noalloc")
     return int(res.value)
 
 
@@ -363,6 +418,56 @@ NOALLOC_MAX_WORDS = 1 << 27  # MMAEMU_XORSUM_NOALLOC_MAX_WORDS
 
 
 def trim_workspace():
-    """Return the current device's cached GEMM workspace (the decoded
-    operands of earlier calls) to the device."""
+    """Return the current device's unused GEMM workspace (cached decoded
+    operands of earlier calls, see set_workspace_cache) to the device."""
     _check(lib().mmaemu_trim_workspace(), "mmaemu_trim_workspace")
+
+
+def set_workspace_cache(enable: bool):
+    """Opt in (or out) of keeping the GEMM workspace between calls on the
+    current device.  Off by default: each GEMM's decoded-operand workspace
+    goes back to the device at the next synchronisation, so the library
+    holds no device memory between calls.  On, repeated GEMMs reuse it and
+    skip the allocation; turning it off trims what is held."""
+    _check(lib().mmaemu_set_workspace_cache(1 if enable else 0), "mmaemu_set_workspace_cache")
+
+
+def workspace_reserved() -> int:
+    """Bytes of device memory the library's workspace pool holds on the
+    current device right now."""
+    v = ctypes.c_size_t(0)
+    _check(lib().mmaemu_workspace_reserved(ctypes.byref(v)), "mmaemu_workspace_reserved")
+    return int(v.value)
+
+
+STATUS_TIMEOUT, STATUS_BOUNDS = 1, 2
+
+
+def device_status(clear: bool = True) -> int:
+    """Bits the kernels recorded on the current device since the last clear
+    (waits for torch's current stream): STATUS_TIMEOUT -- a bounded wait
+    gave up; STATUS_BOUNDS -- the bounds-checking build found an index
+    outside its buffer.  Returns the bits (0: nothing recorded)."""
+    torch = _torch()
+    bits = ctypes.c_uint32(0)
+    set_stream(torch.cuda.current_stream())
+    rc = lib().mmaemu_device_status(1 if clear else 0, ctypes.byref(bits))
+    if rc not in (0, -3, -6):  # OK, ETIMEOUT, EBOUNDS carry the bits
+        _check(rc, "mmaemu_device_status")
+    return int(bits.value)
+
+
+def selftest_wait_timeout(spins: int) -> bool:
+    """Run a kernel whose bounded wait can never complete (nothing ever
+    arrives) with a bound of ``spins`` tries; returns whether it completed
+    (always False).  The timeout is recorded in device_status."""
+    torch = _torch()
+    done = ctypes.c_int(0)
+    set_stream(torch.cuda.current_stream())
+    _check(lib().mmaemu_selftest_wait_timeout(spins, ctypes.byref(done)), "mmaemu_selftest_wait_timeout")
+    return bool(done.value)
+
+
+def bounds_checking() -> bool:
+    """True when the loaded library is the bounds-checking build."""
+    return bool(lib().mmaemu_bounds_checking())

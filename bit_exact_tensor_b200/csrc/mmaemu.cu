@@ -3,16 +3,14 @@
 //
 // Kernels
 //   gemm_kernel   -- D = C + A.B over 16-wide K chunks (ascending, each chunk's
-//                    fp32 result feeding the next), fused per-tile xorsum.
+//                    fp32 result feeding the next), fused per-tile xorsum;
+//                    operand panels decoded once per call (decode_a_kernel,
+//                    decode_b_kernel) and staged by bulk asynchronous copies.
 //   tiles_kernel  -- independent 16x16x16 tiles, one warp per tile.
 //   xorsum_kernel -- XOR of a buffer of 32-bit words.
-// The arithmetic itself is in mmaemu_core.cuh; see the model citations there.
-// Tensor cores are deliberately not used: B200's own MMA arithmetic is not the
-// arithmetic being emulated.  Everything is exact: both kernels keep the
-// exponent-max pass, the carried terms and the write-back in integer (or
-// exact float) steps, and do each product's truncating alignment and signed
-// accumulation in one fused FP64 multiply-add with round-toward-zero, on an
-// integer held in a double's mantissa (see group_products).
+// The arithmetic model and its exact-double formulation are described in
+// mmaemu_core.cuh.  Tensor cores are deliberately not used: B200's own MMA
+// arithmetic is not the arithmetic being emulated.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -25,48 +23,73 @@
 namespace mmaemu {
 
 // ---------------------------------------------------------------------------
+// device status word: bit 0 -- a bounded wait gave up; bit 1 -- a bounds
+// check of the checking build failed (mmaemu_device_status reads it)
+// ---------------------------------------------------------------------------
+__device__ uint32_t g_status;
+constexpr uint32_t STATUS_TIMEOUT = 1u, STATUS_BOUNDS = 2u;
+
+#ifdef MMAEMU_BOUNDS_CHECK
+// checking build: an index outside its buffer is recorded and the access
+// that would use it is skipped
+#define MMAEMU_CHECK(ok, cond)                      \
+  do {                                              \
+    if (!(cond)) {                                  \
+      (ok) = false;                                 \
+      atomicOr(&::mmaemu::g_status, STATUS_BOUNDS); \
+    }                                               \
+  } while (0)
+#else
+#define MMAEMU_CHECK(ok, cond) \
+  do {                         \
+  } while (0)
+#endif
+
+// ---------------------------------------------------------------------------
 // decoded operand panels in shared memory, [k][row] for A and [k][col] for B
 // ---------------------------------------------------------------------------
-// Operand panels of one 16-deep K chunk: the operands as exact doubles for
-// the fused truncate-and-add step of group_products below, the packed
-// negated exponents of the max pass, and the chunk's sign bits per row of A
-// and per column of B.
+// One 16-deep K chunk: the operands as exact doubles (B times 1 + 2^-40),
+// their exponent codes, per row of A and column of B the sign word (A: bit k
+// positive, bit 16+k negative; B: bit k negative, bit 16+k positive; zero,
+// Inf and NaN operands set neither), and a word that is nonzero when the
+// chunk holds an Inf or NaN operand.
 template <int BM, int BN>
 struct __align__(16) Panel {
-  double aV[16][BM];     // A value; zero, Inf and NaN as +-2^-500
-  uint32_t aN2[16][BM];  // (-ea, -ea) packed (ZSENT / NINF / NNAN markers)
-  uint16_t aS[BM];       // bit k: sign of A[m][k]
-  double bV[16][BN];     // B value times (1 + 2^-40); zero, Inf and NaN as +-2^-500
-  int16_t bN2[16][BN];   // -eb (markers as for A)
-  uint16_t bS[BN];       // bit k: sign of B[k][n]
+  double aV[16][BM];
+  uint32_t aQ2[16][BM];  // (q, q): an A code paired with two B codes
+  uint32_t aS[BM];
+  uint32_t aF[4];
+  double bV[16][BN];     // column pairs swizzled in 64-column panels (bslot)
+  int16_t bQ[16][BN];
+  uint32_t bS[BN];
+  uint32_t bF[4];
+  // Slot of column n in a row of bV.  A GEMM thread reads its 8 consecutive
+  // columns as 4 pairs, and the 4 threads of a quarter warp read 4 column
+  // groups 64 bytes apart, which would put groups 0 and 2 (and 1 and 3) on
+  // the same banks; storing pair q of group g at pair q ^ (g & 2) gives each
+  // a bank range of its own.  The tile kernel's 16-column panels keep
+  // natural order (its 4-column groups are conflict-free).
+  static __host__ __device__ constexpr int bslot(int n) {
+    return BN == 64 ? ((n & ~7) | ((((n >> 1) & 3) ^ ((n >> 3) & 2)) << 1) | (n & 1)) : n;
+  }
 };
 
-// Slot of column n (0..BN-1) in a row of bV in the GEMM's panels (the tile
-// kernel's panels keep natural order).  A GEMM thread reads its 8
-// consecutive columns as 4 pairs, and the 4 threads of a quarter warp read
-// 4 column groups 64 bytes apart, which would put groups 0 and 2 (and 1 and
-// 3) on the same banks; storing pair q of group g at pair q ^ (g & 2) gives
-// each a bank range of its own.
-__host__ __device__ constexpr int bv_slot(int n) {
-  return (n & ~7) | ((((n >> 1) & 3) ^ ((n >> 3) & 2)) << 1) | (n & 1);
+template <class PanelT>
+__device__ __forceinline__ int32_t code_a(const PanelT &P, int k, int m) { return lo16(P.aQ2[k][m]); }
+template <class PanelT>
+__device__ __forceinline__ int32_t code_b(const PanelT &P, int k, int n) { return P.bQ[k][n]; }
+template <class PanelT>
+__device__ __forceinline__ bool neg_a(const PanelT &P, int k, int m) { return __double2hiint(P.aV[k][m]) < 0; }
+template <class PanelT>
+__device__ __forceinline__ bool neg_b(const PanelT &P, int k, int n) {
+  return __double2hiint(P.bV[k][PanelT::bslot(n)]) < 0;
 }
 
-// Per-element reads used off the main path (zero-sign rule, Inf/NaN).
-template <int BM, int BN>
-__device__ __forceinline__ int32_t n_a(const Panel<BM, BN> &P, int k, int m) { return lo16(P.aN2[k][m]); }
-template <int BM, int BN>
-__device__ __forceinline__ int32_t n_b(const Panel<BM, BN> &P, int k, int n) { return P.bN2[k][n]; }
-template <int BM, int BN>
-__device__ __forceinline__ bool neg_a(const Panel<BM, BN> &P, int k, int m) { return (P.aS[m] >> k) & 1u; }
-template <int BM, int BN>
-__device__ __forceinline__ bool neg_b(const Panel<BM, BN> &P, int k, int n) { return (P.bS[n] >> k) & 1u; }
-
-// Unroll of the k loops per model and format (measured on the GEMM: 4 for
-// Ampere FP16, 1 for the B200 model, whose 64-bit carry keeps more registers
-// live, else 2).
+// Unroll of the k loops, measured on the GEMM: 4 for the one-stage models;
+// Ampere's two stages spill at 128 registers with any unroll above 1.
 #ifndef MMAEMU_KUNROLL
 template <int MODEL, int FMT>
-constexpr int kUnroll = MODEL == MODEL_AMPERE && FMT == FMT_FP16 ? 4 : MODEL == MODEL_B200 ? 1 : 2;
+constexpr int kUnroll = MODEL == MODEL_AMPERE ? 1 : 4;
 #else
 template <int MODEL, int FMT>
 constexpr int kUnroll = MMAEMU_KUNROLL;
@@ -75,12 +98,7 @@ constexpr int kUnroll = MMAEMU_KUNROLL;
 template <int R, typename T>
 __device__ __forceinline__ void lds_vec(const T *p, T (&v)[R]) {
   static_assert(sizeof(T) == 4, "32-bit elements");
-  if constexpr (R == 8) {
-    const uint4 a = reinterpret_cast<const uint4 *>(p)[0];
-    const uint4 b = reinterpret_cast<const uint4 *>(p)[1];
-    v[0] = (T)a.x; v[1] = (T)a.y; v[2] = (T)a.z; v[3] = (T)a.w;
-    v[4] = (T)b.x; v[5] = (T)b.y; v[6] = (T)b.z; v[7] = (T)b.w;
-  } else if constexpr (R == 4) {
+  if constexpr (R == 4) {
     const uint4 a = reinterpret_cast<const uint4 *>(p)[0];
     v[0] = (T)a.x; v[1] = (T)a.y; v[2] = (T)a.z; v[3] = (T)a.w;
   } else if constexpr (R == 2) {
@@ -91,44 +109,6 @@ __device__ __forceinline__ void lds_vec(const T *p, T (&v)[R]) {
     for (int i = 0; i < R; i++) v[i] = p[i];
   }
 }
-
-// Pass 1 of a group over k in [K0, K0 + KN): nmin (= -e_max) of every output,
-// starting from the carried terms' negated exponents Np (packed pairs).
-template <int FMT, int K0, int KN, int R, int CC, int UNR, class PanelT>
-__device__ __forceinline__ void group_max(const PanelT &P, int rl, int cl, const uint32_t (&Np)[R][CC / 2],
-                                          int32_t (&nmin)[R][CC]) {
-  uint32_t nm2[R][CC / 2];
-#pragma unroll
-  for (int r = 0; r < R; r++)
-#pragma unroll
-    for (int p = 0; p < CC / 2; p++) nm2[r][p] = Np[r][p];
-#pragma unroll UNR
-  for (int k = K0; k < K0 + KN; k++) {
-    uint32_t an2[R], bn2[CC / 2];
-    lds_vec<R>(&P.aN2[k][rl], an2);
-    lds_vec<CC / 2>(reinterpret_cast<const uint32_t *>(&P.bN2[k][cl]), bn2);
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int p = 0; p < CC / 2; p++) nm2[r][p] = vmin2(nm2[r][p], vadd2(an2[r], bn2[p]));
-  }
-#pragma unroll
-  for (int r = 0; r < R; r++)
-#pragma unroll
-    for (int p = 0; p < CC / 2; p++) {
-      uint32_t v = nm2[r][p];
-      if constexpr (kNeedsFloor<FMT>) v = vmin2(v, (uint32_t)NFLOOR | ((uint32_t)NFLOOR << 16));
-      nmin[r][2 * p] = lo16(v);
-      nmin[r][2 * p + 1] = hi16(v);
-    }
-}
-
-__device__ __forceinline__ double fma_rz(double a, double b, double c) {
-  double d;
-  asm("fma.rz.f64 %0, %1, %2, %3;" : "=d"(d) : "d"(a), "d"(b), "d"(c));
-  return d;
-}
-
 template <int R>
 __device__ __forceinline__ void lds_dvec(const double *p, double (&v)[R]) {
   static_assert(R % 2 == 0, "pairs of doubles");
@@ -140,45 +120,115 @@ __device__ __forceinline__ void lds_dvec(const double *p, double (&v)[R]) {
   }
 }
 
-// Pass 2 of a group: add every product's aligned (truncated) magnitude, with
-// its sign, to S (which holds the carried term's contribution), with one
-// fused multiply-add per product.
-// Per output, acc holds (2^52 + 2^51 + L) u on the group's grid u =
-// 2^(e_max - F), with L = S mod 2^32 in its low mantissa bits; every double
-// in [2^52 u, 2^53 u) is a multiple of u, so fma.rz(a, b', acc) -- one
-// rounding, toward zero, of a positive result -- adds floor(a b' / u):
-//  * a positive product adds T = floor(|ab| / u), its truncated magnitude,
-//    because b' = b (1 + 2^-40) moves it by less than the distance to the
-//    next multiple of u (|ab| 2^-40 < 2^(ea+eb+2-40), while |ab| and the grid
-//    points are multiples of 2^(ea+eb-2p) and u >= 2^(ea+eb-F), F < 38);
-//  * a negative product adds -ceil(|ab'| / u) = -T - 1 for the same reason
-//    (|ab'| is never a multiple of u), and a zero stand-in adds 0 or -1 the
-//    same way (T = 0);
-// so the exact sum is L plus the number of negative products, which is the
-// popcount of the XOR of the row's and the column's sign bits over the
-// group.  L stays far inside the 51-bit field, and the low 32 bits of acc
-// give the sum modulo 2^32 (the sums here fit in int32).
-// The exponent field is 1075 - F - nmin, formed modulo 2^32: the marker
-// values of nmin (ZSENT, NINF and sums with them) are multiples of 2^12
-// plus a real n, so they wrap to a valid grid; such a group has no nonzero
-// term (or is overwritten as Inf/NaN), and every product of a zero stand-in
-// (below 2^-371) truncates to zero on it.
-template <int F, int K0, int KN, int R, int CC, int UNR, int BM, int BN>
-__device__ __forceinline__ void group_products(const Panel<BM, BN> &P, int rl, int cl,
-                                               const int32_t (&nmin)[R][CC], int32_t (&S)[R][CC]) {
-  double acc[R][CC];
-  constexpr uint32_t HI0 = ((uint32_t)(1075 - F) << 20) | 0x80000u;
+__device__ __forceinline__ double fma_rz(double a, double b, double c) {
+  double d;
+  asm("fma.rz.f64 %0, %1, %2, %3;" : "=d"(d) : "d"(a), "d"(b), "d"(c));
+  return d;
+}
+__device__ __forceinline__ double fma_rn(double a, double b, double c) {
+  double d;
+  asm("fma.rn.f64 %0, %1, %2, %3;" : "=d"(d) : "d"(a), "d"(b), "d"(c));
+  return d;
+}
+// truncation to 24 significant bits (toward zero) of a normal double, zero,
+// Inf or NaN with an all-ones high word
+__device__ __forceinline__ double mask24(double v) {
+  return __hiloint2double(__double2hiint(v), __double2loint(v) & (int)0xE0000000u);
+}
+// 2^k as a double (normal k)
+__host__ __device__ constexpr double pow2d(int k) {
+  double r = 1.0;
+  for (; k > 0; k--) r *= 2.0;
+  for (; k < 0; k++) r *= 0.5;
+  return r;
+}
+
+// High word of a group's base 1.5 * 2^52 * u, u = 2^(e_max - F), from the
+// packed code pair nm (lane 0 for the even output, lane 1 for the odd one):
+// e_max = 1024 - nm / 16 gives the exponent field 2099 - F - nm / 16.  For
+// the odd output the low lane's code is subtracted from the low mantissa
+// bits as well (it is below 2^15, so it never borrows from the exponent):
+// that base is a little below 1.5 * 2^52 u, still a multiple of u in the
+// same binade, and the same value is used to add and to subtract it.
+template <int F, int ODD>
+__device__ __forceinline__ uint32_t base_hi(uint32_t nm) {
+  constexpr uint32_t KHI = ((uint32_t)(2099 - F) << 20) | 0x80000u;
+  return ODD ? KHI - nm : KHI + nm * 0xFFFF0000u;
+}
+
+// Carried terms' codes, two outputs per word, from the top 16 bits of their
+// doubles: unchecked (value as is) ncode(e) = (2047 - field) * 16 directly;
+// checked (value times 2^s, field >= 1024 for every nonzero value) the low
+// ten exponent bits give ncode(e) - 16 s, and the offset is added later.
+template <bool CHK, int R, int CC>
+__device__ __forceinline__ void carry_codes(const double (&X)[R][CC], uint32_t (&c2)[R][CC / 2]) {
 #pragma unroll
   for (int r = 0; r < R; r++)
 #pragma unroll
-    for (int c = 0; c < CC; c++)
-      acc[r][c] = __hiloint2double((int)(HI0 - ((uint32_t)nmin[r][c] << 20)), S[r][c]);
-  // 8-column groups (GEMM) are stored with their pairs swizzled (bv_slot);
-  // 4-column groups (tile kernel) in natural order, which is conflict-free
+    for (int p = 0; p < CC / 2; p++) {
+      const uint32_t x = __byte_perm((uint32_t)__double2hiint(X[r][2 * p]), (uint32_t)__double2hiint(X[r][2 * p + 1]),
+                                     0x7632);
+      c2[r][p] = ~x & (CHK ? 0x3FF03FF0u : 0x7FF07FF0u);
+    }
+}
+
+// Group codes: from the carried terms' codes (carry_codes; checked codes get
+// their offset to ncode and the -133 floor, which changes nothing but BF16)
+// down to the minimum over the group's products, qa + qb for k in [K0, K0 +
+// KN), two outputs per packed add-and-min: nm becomes ncode(e_max).
+template <int FMT, bool CHK, int KN, int UNR, int R, int C2, class PanelT>
+__device__ __forceinline__ void group_codes(const PanelT &P, int rl, int cl, int K0, uint32_t (&nm)[R][C2],
+                                            int SIN) {
+  constexpr int CC = 2 * C2;
+  if constexpr (CHK) {
+#pragma unroll
+    for (int r = 0; r < R; r++)
+#pragma unroll
+      for (int p = 0; p < C2; p++)
+        nm[r][p] = vmin2(vadd2(nm[r][p], (uint32_t)(16 * SIN) * 0x10001u), pair16(FLOOR_CODE, FLOOR_CODE));
+  } else {
+    static_assert(!kNeedsFloor<FMT>, "BF16 runs checked");
+  }
+#pragma unroll UNR
+  for (int i = 0; i < KN; i++) {
+    const int k = K0 + i;
+    uint32_t an2[R], bn2[C2];
+    lds_vec<R>(&P.aQ2[k][rl], an2);
+    lds_vec<C2>(reinterpret_cast<const uint32_t *>(&P.bQ[k][cl]), bn2);
+#pragma unroll
+    for (int r = 0; r < R; r++)
+#pragma unroll
+      for (int p = 0; p < C2; p++) nm[r][p] = vmin2(vadd2(an2[r], bn2[p]), nm[r][p]);
+  }
+  (void)CC;
+}
+
+// Accumulators of one group: base plus the count of negative terms, then the
+// carried value (X on entry) added like a product, times the same 1 + 2^-40.
+template <int F, int R, int CC, int C2, class PanelT>
+__device__ __forceinline__ void group_start(const PanelT &P, int rl, int cl, double (&X)[R][CC],
+                                            const uint32_t (&nm)[R][C2], double SKEW, uint32_t GM) {
+  uint32_t sa[R], sb[CC];
+  lds_vec<R>(&P.aS[rl], sa);
+  lds_vec<CC>(&P.bS[cl], sb);
+#pragma unroll
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int c = 0; c < CC; c++) {
+      const uint32_t hi = (c & 1) ? base_hi<F, 1>(nm[r][c / 2]) : base_hi<F, 0>(nm[r][c / 2]);
+      const uint32_t cnt = __popc(sa[r] & sb[c] & GM) + ((uint32_t)__double2hiint(X[r][c]) >> 31);
+      X[r][c] = fma_rz(X[r][c], SKEW, __hiloint2double((int)hi, (int)cnt));
+    }
+}
+
+// One round-toward-zero fused multiply-add per product of k in [K0, K0+KN).
+template <int KN, int UNR, int R, int CC, class PanelT>
+__device__ __forceinline__ void group_products(const PanelT &P, int rl, int cl, int K0, double (&X)[R][CC]) {
   static_assert(CC == 8 || CC == 4, "column groups of 8 or 4");
   const int sw = (cl >> 3) & 2;
 #pragma unroll UNR
-  for (int k = K0; k < K0 + KN; k++) {
+  for (int i = 0; i < KN; i++) {
+    const int k = K0 + i;
     double a[R], b[CC];
     lds_dvec<R>(&P.aV[k][rl], a);
     if constexpr (CC == 8) {
@@ -194,86 +244,64 @@ __device__ __forceinline__ void group_products(const Panel<BM, BN> &P, int rl, i
 #pragma unroll
     for (int c = 0; c < CC; c++)
 #pragma unroll
-      for (int r = 0; r < R; r++) acc[r][c] = fma_rz(a[r], b[c], acc[r][c]);
+      for (int r = 0; r < R; r++) X[r][c] = fma_rz(a[r], b[c], X[r][c]);
   }
-  constexpr uint32_t GM = ((1u << KN) - 1u) << K0;
-  uint32_t sa[R], sb[CC];
-#pragma unroll
-  for (int r = 0; r < R; r++) sa[r] = P.aS[rl + r];
-#pragma unroll
-  for (int c = 0; c < CC; c++) sb[c] = P.bS[cl + c];
+}
+
+// exact group value: accumulator minus its base
+template <int F, int R, int CC>
+__device__ __forceinline__ double group_value(const double (&X)[R][CC], const uint32_t (&nm)[R][CC / 2], int r,
+                                              int c) {
+  uint32_t hi;
+  constexpr uint32_t KHI = ((uint32_t)(2099 - F) << 20) | 0x80000u;
+  if (c & 1) asm volatile("sub.u32 %0, %1, %2;" : "=r"(hi) : "r"(KHI), "r"(nm[r][c / 2]));
+  else asm volatile("mad.lo.u32 %0, %1, %2, %3;" : "=r"(hi) : "r"(nm[r][c / 2]), "r"(0xFFFF0000u), "r"(KHI));
+  return X[r][c] - __hiloint2double((int)hi, 0);
+}
+
+// Checked states below 2^-126 in magnitude: truncate onto the fp32 subnormal
+// grid 2^-149 (a value that truncates to zero keeps the sign of the sum), and
+// give the carried term the exponent -126 of an fp32 subnormal.  c2 holds the
+// carried codes of carry_codes<true>: normal scaled fp32 values give 16..4064,
+// zero 16368, Inf and NaN 0, fp32 subnormals lie strictly between.
+template <int R, int CC>
+__device__ __forceinline__ void subnormal_states(double (&X)[R][CC], uint32_t (&c2)[R][CC / 2], uint32_t &dneg0) {
+  uint32_t t = 0xFFFFFFFFu;
 #pragma unroll
   for (int r = 0; r < R; r++)
 #pragma unroll
-    for (int c = 0; c < CC; c++)
-      S[r][c] = (int32_t)((uint32_t)__double2loint(acc[r][c]) + __popc((sa[r] ^ sb[c]) & GM));
-}
-
-// One accumulation group with a carried term in the state form (Np, X):
-// returns S (exact signed sum of the aligned terms) and nmin (= -e_max).
-template <int FMT, int F, int K0, int KN, int R, int CC, int UNR, class PanelT>
-__device__ __forceinline__ void group_sum(const PanelT &P, int rl, int cl, const uint32_t (&Np)[R][CC / 2],
-                                          const int32_t (&X)[R][CC], int32_t (&nmin)[R][CC], int32_t (&S)[R][CC]) {
-  group_max<FMT, K0, KN, R, CC, UNR>(P, rl, cl, Np, nmin);
-  constexpr int CSH = 30 - F;  // the state's significand sits at bits 30..7
+    for (int p = 0; p < CC / 2; p++) t = vminu2(t, vadd2(c2[r][p], pair16(-4065, -4065)));
+  if ((t & 0xFFFFu) >= 12303u && (t >> 16) >= 12303u) return;
+  // rare: unrolled, so that the states stay in registers
 #pragma unroll
   for (int r = 0; r < R; r++)
 #pragma unroll
     for (int c = 0; c < CC; c++) {
-      const int32_t nc = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
-      // ones' complement -> exact: ~(M >> d) + 1 = -(M >> d)
-      S[r][c] = shr_s32(X[r][c], (uint32_t)(nc - nmin[r][c] + CSH)) + (int32_t)((uint32_t)X[r][c] >> 31);
+      const uint32_t code = (c & 1) ? (c2[r][c / 2] >> 16) : (c2[r][c / 2] & 0xFFFFu);
+      if (code <= 4064u || code >= 16368u) continue;
+      const uint32_t bit = 1u << (r * CC + c);
+      const double x = X[r][c];
+      constexpr double TO_Q = pow2d(-(S_WB - 149)), FROM_Q = pow2d(S_WB - 149);
+    const double q = trunc(fabs(x) * TO_Q);  // |value| 2^149
+      if (q == 0.0) {
+        X[r][c] = 0.0;
+        dneg0 = x < 0.0 ? (dneg0 | bit) : (dneg0 & ~bit);
+      } else {
+        X[r][c] = copysign(q * FROM_Q, x);
+        const uint32_t sub = (uint32_t)(SUBN_CODE - 16 * S_WB);
+        c2[r][c / 2] = (c & 1) ? ((c2[r][c / 2] & 0xFFFFu) | (sub << 16)) : ((c2[r][c / 2] & 0xFFFF0000u) | sub);
+      }
     }
-  group_products<F, K0, KN, R, CC, UNR>(P, rl, cl, nmin, S);
 }
-
-// normalise a sum to the state form: X with its leading bit at bit 30 (in
-// ones' complement when negative) and n = -(exponent of the leading bit).
-// S == 0 gives X == 0 (its n is meaningless and is fixed by the caller).
-__device__ __forceinline__ uint32_t msb_pos(uint32_t x) {  // -1 (all ones) for x == 0
-  uint32_t p;
-  asm("bfind.u32 %0, %1;" : "=r"(p) : "r"(x));
-  return p;
-}
-template <int F>
-__device__ __forceinline__ void to_state(int32_t s, int32_t nmin, int32_t &n, int32_t &X, uint32_t mask) {
-  const uint32_t mag = (uint32_t)(s < 0 ? -s : s);
-  const int32_t p = (int32_t)msb_pos(mag);
-  const uint32_t M = shl_u32(mag, (uint32_t)(30 - p));
-  n = nmin + F - p;  // the leading bit is worth 2^(e_max - F + p)
-  X = (int32_t)((M & mask) ^ (uint32_t)(s >> 31));
-}
-// the same for a sum that may need 33 bits (F = 25)
-template <int F>
-__device__ __forceinline__ void to_state64(int64_t s, int32_t nmin, int32_t &n, int32_t &X, uint32_t mask) {
-  const uint64_t mag = (uint64_t)(s < 0 ? -s : s);
-  const int32_t p = 63 - __clzll((long long)mag);  // -1 for 0
-  const uint32_t M = p > 30 ? (uint32_t)(mag >> (p - 30)) : shl_u32((uint32_t)mag, (uint32_t)(30 - p));
-  n = nmin + F - p;
-  X = (int32_t)((M & mask) ^ (uint32_t)(s < 0 ? 0xFFFFFFFFu : 0u));
-}
-
-// Zero tests of panel operands (the zero-sign rule needs them).
-template <class PanelT>
-__device__ __forceinline__ bool zero_a(const PanelT &P, int k, int m) { return n_a(P, k, m) == ZSENT; }
-template <class PanelT>
-__device__ __forceinline__ bool zero_b(const PanelT &P, int k, int n) { return n_b(P, k, n) == ZSENT; }
 
 // Special-value outcome of each output of an R x CC block whose chunk holds
 // Inf or NaN somewhere in its A or B panel: 2 bits per output (0 none, 1 NaN,
-// 2 +Inf, 3 -Inf).  c_nan / c_infp / c_infn flag outputs whose incoming value
-// is NaN / +Inf / -Inf.  Kept out of line: it is rare and would otherwise
-// crowd the registers of the main path.
+// 2 +Inf, 3 -Inf).  Any NaN, or Inf x 0, gives NaN; infinities of both signs
+// (including an infinite incoming value) give NaN, of one sign that Inf.
+// c_nan / c_infp / c_infn flag outputs whose incoming value is NaN / +Inf /
+// -Inf.  Kept out of line: it is rare.
 template <int R, int CC, class PanelT>
-__device__ __noinline__ uint64_t special_codes(const PanelT *P, int rl, int cl, uint32_t c_nan, uint32_t c_infp,
-                                               uint32_t c_infn);
-template <int R, int CC, class PanelT>
-__device__ __forceinline__ uint64_t special_codes(const PanelT &P, int rl, int cl, uint32_t c_nan, uint32_t c_infp,
-                                                  uint32_t c_infn) {
-  return special_codes<R, CC>(&P, rl, cl, c_nan, c_infp, c_infn);
-}
-template <int R, int CC, class PanelT>
-__device__ __noinline__ uint64_t special_codes(const PanelT *P, int rl, int cl, uint32_t c_nan, uint32_t c_infp,
+__device__ __forceinline__ uint64_t special_codes(const PanelT *P, int rl, int cl, uint32_t c_nan, uint32_t c_infp,
                                                uint32_t c_infn) {
   uint64_t codes = 0;
 #pragma unroll 1
@@ -282,11 +310,11 @@ __device__ __noinline__ uint64_t special_codes(const PanelT *P, int rl, int cl, 
     bool nan = (c_nan >> o) & 1u, ip = (c_infp >> o) & 1u, in = (c_infn >> o) & 1u;
 #pragma unroll 1
     for (int k = 0; k < 16; k++) {
-      const int32_t an = n_a(*P, k, rl + r), bn = n_b(*P, k, cl + c);
-      if (an == NNAN || bn == NNAN) {
+      const int32_t aq = code_a(*P, k, rl + r), bq = code_b(*P, k, cl + c);
+      if (aq == QNAN || bq == QNAN) {
         nan = true;
-      } else if (an == NINF || bn == NINF) {
-        if (an == ZSENT || bn == ZSENT) nan = true;
+      } else if (aq == QINF || bq == QINF) {
+        if (aq == QZ || bq == QZ) nan = true;
         else if (neg_a(*P, k, rl + r) != neg_b(*P, k, cl + c)) in = true;
         else ip = true;
       }
@@ -297,372 +325,196 @@ __device__ __noinline__ uint64_t special_codes(const PanelT *P, int rl, int cl, 
   return codes;
 }
 
-// One 16-deep K chunk for an R x CC block of outputs at panel row rl, col cl,
-// updating the accumulator state (Np, X, dneg0) in place.
-//   Np    -- n of adjacent output pairs, packed
-//   X     -- significands (see mmaemu_core.cuh)
-//   dneg0 -- bit r*CC+c set when that output's state is -0
-template <int MODEL, int FMT, int R, int CC, class PanelT>
-__device__ __forceinline__ void mma_chunk(const PanelT &P, int rl, int cl, uint32_t (&Np)[R][CC / 2],
-                                          int32_t (&X)[R][CC], uint32_t &dneg0, bool panel_special) {
+// zero-sign rule for a zero sum: -0 only when the incoming value is -0 and
+// all 16 products are zeros of negative sign
+template <class PanelT>
+__device__ __forceinline__ bool all_products_negative_zero(const PanelT *P, int m, int n) {
+#pragma unroll 1
+  for (int k = 0; k < 16; k++) {
+    const bool zero = code_a(*P, k, m) == QZ || code_b(*P, k, n) == QZ;
+    if (!zero || neg_a(*P, k, m) == neg_b(*P, k, n)) return false;
+  }
+  return true;
+}
+
+// One 16-deep K chunk for an R x CC block of outputs, updating the states X
+// in place.  CHK selects the checked form (values times 2^896; overflow,
+// underflow, Inf and NaN handled); the unchecked form serves FP16 / E4M3
+// states that cannot leave the normal fp32 range (see init_states).
+//   dneg0      -- bit r*CC+c set when that output's state is -0 (stored +0)
+//   to_checked -- set by the unchecked form when an Inf/NaN operand made a
+//                 result infinite or NaN: the caller scales the states and
+//                 continues checked
+// Ampere's two stages run as a loop over one copy of the group code, so
+// that the compiler cannot interleave them (which costs registers).
+template <int MODEL, int FMT, bool CHK, int R, int CC, class PanelT>
+__device__ __forceinline__ void mma_chunk(const PanelT &P, int rl, int cl, double (&X)[R][CC], uint32_t &dneg0,
+                                          bool panel_special, bool &to_checked) {
   constexpr int F = ModelT<MODEL>::F;
+  constexpr int KN = ModelT<MODEL>::STAGE1;  // group size
   constexpr int UNR = kUnroll<MODEL, FMT>;
+  constexpr int NST = MODEL == MODEL_AMPERE ? 2 : 1;
   static_assert(R * CC <= 32 && CC % 2 == 0, "per-output masks hold 32 outputs");
-  // with 24 or more fraction bits the grid would see state bits below the
-  // fp32 value's 24: keep bits 0..6 clear
-  constexpr uint32_t XMASK = F >= 24 ? 0x7FFFFF80u : 0x7FFFFFFFu;
+  constexpr double SKEW_PLAIN = 1.0 + pow2d(-40), SKEW_WB = SKEW_PLAIN * pow2d(-S_WB),
+                   SKEW_HO = SKEW_PLAIN * pow2d(-S_HO);
 
   // kinds of the incoming values, needed only when A/B hold Inf or NaN
   uint32_t c_nan = 0, c_infp = 0, c_infn = 0;
-  if (panel_special) {
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int c = 0; c < CC; c++) {
-        const int32_t n = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
-        const uint32_t bit = 1u << (r * CC + c);
-        if (n == STATE_NAN) c_nan |= bit;
-        if (n == STATE_INF) {
-          if (X[r][c] < 0) c_infn |= bit;
-          else c_infp |= bit;
-        }
-      }
-  }
-
-  int32_t S[R][CC], nmin[R][CC];
-  if constexpr (MODEL == MODEL_AMPERE) {
-    // stage 1: {C, P[1..8]}
-    group_sum<FMT, F, 0, 8, R, CC, UNR>(P, rl, cl, Np, X, nmin, S);
-    // hand-over: the stage-1 sum as a 24-bit term (the state form keeps extra
-    // low bits, but stage 2 shifts it right by at least 7, which truncates
-    // them exactly like the normalisation would); a zero sum adds no term
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int p = 0; p < CC / 2; p++) {
-        int32_t n0, n1;
-        to_state<F>(S[r][2 * p], nmin[r][2 * p], n0, X[r][2 * p], 0x7FFFFFFFu);
-        to_state<F>(S[r][2 * p + 1], nmin[r][2 * p + 1], n1, X[r][2 * p + 1], 0x7FFFFFFFu);
-        Np[r][p] = pack16(S[r][2 * p] ? n0 : ZSENT, S[r][2 * p + 1] ? n1 : ZSENT);
-      }
-    // stage 2: {S1, P[9..16]}
-    group_sum<FMT, F, 8, 8, R, CC, UNR>(P, rl, cl, Np, X, nmin, S);
-  } else if constexpr (kWideSum<MODEL>) {
-    // one stage {C, P[1..16]}: the products here, C in the write-back
-    group_max<FMT, 0, 16, R, CC, UNR>(P, rl, cl, Np, nmin);
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int c = 0; c < CC; c++) S[r][c] = 0;
-    group_products<F, 0, 16, R, CC, UNR>(P, rl, cl, nmin, S);
-  } else {
-    // one stage: {C, P[1..16]}
-    group_sum<FMT, F, 0, 16, R, CC, UNR>(P, rl, cl, Np, X, nmin, S);
-  }
-
-  // toward-zero write-back into the state (the fp32 value is its top 24 bits)
-  bool any_rare = false;
-#pragma unroll
-  for (int r = 0; r < R; r++)
-#pragma unroll
-    for (int p = 0; p < CC / 2; p++) {
-      int32_t n0, n1;
-      if constexpr (kWideSum<MODEL>) {
-        // add the carried state (ones' complement alignment, as group_sum)
-        // to the products in 64 bits
-        int32_t nn[2];
-#pragma unroll
-        for (int q = 0; q < 2; q++) {
-          const int c = 2 * p + q;
-          const int32_t nc = q ? hi16(Np[r][p]) : lo16(Np[r][p]);
-          const int32_t carry = shr_s32(X[r][c], (uint32_t)(nc - nmin[r][c] + 30 - F)) +
-                                (int32_t)((uint32_t)X[r][c] >> 31);
-          to_state64<F>((int64_t)S[r][c] + carry, nmin[r][c], nn[q], X[r][c], XMASK);
-        }
-        n0 = nn[0];
-        n1 = nn[1];
-      } else {
-        to_state<F>(S[r][2 * p], nmin[r][2 * p], n0, X[r][2 * p], XMASK);
-        to_state<F>(S[r][2 * p + 1], nmin[r][2 * p + 1], n1, X[r][2 * p + 1], XMASK);
-      }
-      Np[r][p] = pack16(n0, n1);
-      // zero (X == 0 exactly when S == 0), or the exponent outside [-126, 127]
-      any_rare = any_rare || X[r][2 * p] == 0 || (uint32_t)(n0 + 127) > 253u || X[r][2 * p + 1] == 0 ||
-                 (uint32_t)(n1 + 127) > 253u;
-    }
-  uint32_t rare = 0;
-  if (any_rare) {
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int c = 0; c < CC; c++) {
-        const int32_t n0 = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
-        if (X[r][c] == 0 || (uint32_t)(n0 + 127) > 253u) rare |= 1u << (r * CC + c);
-      }
-  }
-  dneg0 &= rare;  // every ordinary result is nonzero
-
-  if (rare) {
-    // Only the new state is used here: S == 0 left X == 0, and for S != 0
-    // X ^ sgn = (|S| << clz) >> 1 with n = -(exponent of the leading bit).
+  if (CHK && panel_special) {
 #pragma unroll
     for (int r = 0; r < R; r++)
 #pragma unroll
       for (int c = 0; c < CC; c++) {
         const uint32_t bit = 1u << (r * CC + c);
-        if (!(rare & bit)) continue;
-        const int32_t x0 = X[r][c];
-        const int32_t n0 = (c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]);
-        const uint32_t sg = (uint32_t)(x0 >> 31);
-        int32_t n;
-        int32_t x;
-        bool negz = false;
-        if (x0 == 0) {
-          // zero-sign rule: -0 only when C and all 16 products are -0
-          bool neg = (dneg0 & bit) != 0;
-          for (int k = 0; k < 16 && neg; k++) {
-            const bool zero = zero_a(P, k, rl + r) || zero_b(P, k, cl + c);
-            neg = zero && neg_a(P, k, rl + r) != neg_b(P, k, cl + c);
-          }
-          n = ZSENT;
-          x = neg ? -1 : 0;
-          negz = neg;
-        } else if (n0 <= STATE_NAN + 50) {  // a NaN carried in
-          n = STATE_NAN;
-          x = 0x40000000;
-        } else if (n0 < -127) {  // exponent above 127: overflow to infinity
-          n = STATE_INF;
-          x = (int32_t)(0x40000000u ^ sg);
-        } else {
-          // below 2^-126: truncate onto the subnormal grid 2^-149, i.e.
-          // q = floor(|S| 2^(e_max - F + 149)) = ((X ^ sgn) >> (n - 119))
-          const uint32_t q = shr_u32((uint32_t)x0 ^ sg, (uint32_t)(n0 - 119));
-          if (q == 0) {
-            n = ZSENT;
-            x = (int32_t)sg;
-            negz = sg != 0;
+        if (isnan(X[r][c])) c_nan |= bit;
+        else if (isinf(X[r][c])) (X[r][c] < 0.0 ? c_infn : c_infp) |= bit;
+      }
+  }
+  uint32_t nm[R][CC / 2];
+  carry_codes<CHK>(X, nm);
+  if constexpr (CHK) subnormal_states(X, nm, dneg0);
+#pragma unroll 1
+  for (int st = 0; st < NST; st++) {
+    const int sin = !CHK ? 0 : st ? S_HO : S_WB;
+    const double skew = !CHK ? SKEW_PLAIN : st ? SKEW_HO : SKEW_WB;
+    const uint32_t gm = (NST == 1 ? 0xFFFFu : st ? 0xFF00u : 0x00FFu) * 0x10001u;
+    const int k0 = KN * st;
+    group_codes<FMT, CHK, KN, UNR>(P, rl, cl, k0, nm, sin);
+    group_start<F>(P, rl, cl, X, nm, skew, gm);
+    group_products<KN, UNR>(P, rl, cl, k0, X);
+    if (st + 1 < NST) {
+      // hand-over: the stage-1 value truncated to 24 bits, exponent unbounded
+      // (checked: times 2^512, formed in one exact fused multiply-add); a
+      // zero stage adds nothing
+#pragma unroll
+      for (int r = 0; r < R; r++)
+#pragma unroll
+        for (int c = 0; c < CC; c++) {
+          if constexpr (CHK) {
+            constexpr double UP_HO = pow2d(S_HO);
+            const uint32_t hi = (c & 1) ? base_hi<F, 1>(nm[r][c / 2]) : base_hi<F, 0>(nm[r][c / 2]);
+            X[r][c] = mask24(fma_rn(X[r][c], UP_HO, -__hiloint2double((int)(hi + ((uint32_t)S_HO << 20)), 0)));
           } else {
-            n = 126;
-            x = (int32_t)((q << 7) ^ sg);
+            X[r][c] = mask24(group_value<F>(X, nm, r, c));
           }
         }
-        X[r][c] = x;
-        Np[r][c / 2] = (c & 1) ? pack16(lo16(Np[r][c / 2]), n) : pack16(n, hi16(Np[r][c / 2]));
-        dneg0 = negz ? (dneg0 | bit) : (dneg0 & ~bit);
-      }
-  }
-
-  // special values: NaN anywhere or Inf x 0 -> NaN; Inf of one sign -> that
-  // Inf; both signs -> NaN
-  if (panel_special) {
-    const uint64_t codes = special_codes<R, CC>(P, rl, cl, c_nan, c_infp, c_infn);
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int c = 0; c < CC; c++) {
-        const uint32_t code = (uint32_t)(codes >> (2 * (r * CC + c))) & 3u;
-        if (code == 0u) continue;
-        const int32_t n = code == 1u ? STATE_NAN : STATE_INF;
-        X[r][c] = code == 3u ? (int32_t)0xBFFFFFFFu : 0x40000000;
-        Np[r][c / 2] = (c & 1) ? pack16(lo16(Np[r][c / 2]), n) : pack16(n, hi16(Np[r][c / 2]));
-        dneg0 &= ~(1u << (r * CC + c));
-      }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Float-assisted chunk (FP16 and E4M3 inputs).  The accumulator state is the
-// fp32 value D itself (plus n = -e(D) in packed pairs), and the steps around
-// the integer group sums run on the conversion and FMA units:
-//  * a carried fp32 value c contributes trunc(c 2^(F - e_max)): one exact
-//    multiply by a power of two and one toward-zero conversion to int;
-//  * cvt.rz.f32.s32(S) is S truncated to 24 significant bits with its sign
-//    and exponent -- the Ampere stage hand-over (W = 24) and the fp32
-//    write-back, which is that float times 2^(e_max - F).
-//
-// Range.  A thread takes this path only if every C value it starts from is
-// +-0 or of magnitude in [2^-60, 2^63).  FP16 products are below 2^32 and
-// E4M3 products below 2^18, so over any K < 2^31 a running value stays below
-// 2^64 (truncation never rounds up).  A group with a nonzero product has
-// e_max >= -28, so a nonzero sum is at least one unit of the grid
-// 2^(e_max - F) >= 2^-52; without one, the sum is the carried value itself.
-// Hence every D is +-0 or normal with n = -e(D) in [-63, 60]: the write-back
-// can neither overflow nor underflow, and every power of two formed below
-// is a normal float.  Inf/NaN operands hand the thread to the integer path.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ float i2f_rz(int32_t s) {
-  float f;
-  asm("cvt.rz.f32.s32 %0, %1;" : "=f"(f) : "r"(s));
-  return f;
-}
-__device__ __forceinline__ int32_t f2i_rz(float f) {
-  int32_t r;
-  asm("cvt.rzi.s32.f32 %0, %1;" : "=r"(r) : "f"(f));
-  return r;
-}
-// biased exponent field of a float (0 for zero)
-__device__ __forceinline__ int32_t exp_field(float f) { return (int32_t)((__float_as_uint(f) << 1) >> 24); }
-// 2^k as a float for k in [-126, 127] (one IMAD)
-__device__ __forceinline__ float pow2f(int32_t k) { return __uint_as_float((uint32_t)k * 0x800000u + 0x3F800000u); }
-
-// the path's range of accumulator magnitudes: [2^-FAST_NMAX, 2^FAST_EMAX)
-constexpr int FAST_NMAX = 60, FAST_EMAX = 63;
-// BF16 products and sums reach exponents far outside the float range
-template <int FMT> constexpr bool kFloatAssisted = FMT != FMT_BF16;
-// Ampere stage hand-over: S1 is carried as g1 = S1_24 2^(-HX - e_max1) and
-// scaled by 2^(HX + e_max2) in stage 2.  With HX = 42 both factors stay
-// normal for e_max in [-60, 63], and when S1 == 0 (its n then reads
-// e_max1 + 150 instead of a zero marker) the stage-2 factor, if that n
-// becomes stage 2's maximum, is a finite float: the zero carry stays zero.
-constexpr int HX = 42;
-
-template <int MODEL, int FMT, int R, int CC, class PanelT>
-__device__ __forceinline__ void mma_chunk_fast(const PanelT &P, int rl, int cl, uint32_t (&Np)[R][CC / 2],
-                                               uint32_t (&V)[R][CC], uint32_t &dneg0, bool panel_special,
-                                               bool &to_integer) {
-  constexpr int F = ModelT<MODEL>::F;
-  static_assert(FMT != FMT_BF16, "BF16 exponents leave the float range");
-  int32_t S[R][CC], nmin[R][CC];
-  constexpr int KN1 = MODEL == MODEL_AMPERE ? 8 : 16;
-  constexpr bool WIDE = kWideSum<MODEL>;
-  constexpr int UNR = kUnroll<MODEL, FMT>;
-  // first (or only) group: carried D plus products (the carried term is
-  // added in the write-back when the sum may need 33 bits)
-  group_max<FMT, 0, KN1, R, CC, UNR>(P, rl, cl, Np, nmin);
-#pragma unroll
-  for (int r = 0; r < R; r++)
-#pragma unroll
-    for (int c = 0; c < CC; c++)
-      S[r][c] = WIDE ? 0 : f2i_rz(__uint_as_float(V[r][c]) * pow2f(F + nmin[r][c]));
-  group_products<F, 0, KN1, R, CC, UNR>(P, rl, cl, nmin, S);
-  if constexpr (MODEL == MODEL_AMPERE) {
-    // hand-over: the stage-1 sum truncated to 24 bits; a zero sum needs no
-    // marker (see HX): its n exceeds every nonzero product's n (<= 28)
-    float g1[R][CC];
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int p = 0; p < CC / 2; p++) {
-        int32_t n1[2];
-#pragma unroll
-        for (int q = 0; q < 2; q++) {
-          const int c = 2 * p + q;
-          const float f1 = i2f_rz(S[r][c]);
-          n1[q] = nmin[r][c] + (F + 127) - exp_field(f1);
-          g1[r][c] = f1 * pow2f(-HX - nmin[r][c]);
-        }
-        Np[r][p] = pack16(n1[0], n1[1]);
-      }
-    group_max<FMT, 8, 8, R, CC, UNR>(P, rl, cl, Np, nmin);
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int c = 0; c < CC; c++) S[r][c] = f2i_rz(g1[r][c] * pow2f(nmin[r][c] + HX));
-    group_products<F, 8, 8, R, CC, UNR>(P, rl, cl, nmin, S);
-  }
-
-  // write-back: D = cvt.rz(S) 2^(e_max - F), exact (D is normal)
-  bool any_zero = false;
-#pragma unroll
-  for (int r = 0; r < R; r++)
-#pragma unroll
-    for (int p = 0; p < CC / 2; p++) {
-      int32_t nn[2];
-#pragma unroll
-      for (int q = 0; q < 2; q++) {
-        const int c = 2 * p + q;
-        float f2;
-        if constexpr (WIDE) {
-          const int64_t s64 = (int64_t)S[r][c] + f2i_rz(__uint_as_float(V[r][c]) * pow2f(F + nmin[r][c]));
-          asm("cvt.rz.f32.s64 %0, %1;" : "=f"(f2) : "l"(s64));
-          S[r][c] = s64 != 0;  // only the zero test below reads S
-        } else {
-          f2 = i2f_rz(S[r][c]);
-        }
-        nn[q] = nmin[r][c] + (F + 127) - exp_field(f2);
-        V[r][c] = __float_as_uint(f2 * pow2f(-F - nmin[r][c]));
-        any_zero = any_zero || S[r][c] == 0;
-      }
-      Np[r][p] = pack16(nn[0], nn[1]);
+      carry_codes<CHK>(X, nm);
     }
-  uint32_t zero = 0;
-  if (any_zero) {
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int c = 0; c < CC; c++) {
-        if (S[r][c] != 0) continue;
-        const uint32_t bit = 1u << (r * CC + c);
-        zero |= bit;
-        // zero-sign rule: -0 only when C and all 16 products are -0
-        bool neg = (dneg0 & bit) != 0;
-        for (int k = 0; k < 16 && neg; k++) {
-          const bool z = zero_a(P, k, rl + r) || zero_b(P, k, cl + c);
-          neg = z && neg_a(P, k, rl + r) != neg_b(P, k, cl + c);
-        }
-        V[r][c] = neg ? 0x80000000u : 0u;
-        Np[r][c / 2] = (c & 1) ? pack16(lo16(Np[r][c / 2]), ZSENT) : pack16(ZSENT, hi16(Np[r][c / 2]));
-        dneg0 = neg ? (dneg0 | bit) : (dneg0 & ~bit);
-      }
   }
-  dneg0 &= zero;
-
-  // Inf/NaN operands (the incoming values are finite on this path)
-  if (panel_special) {
-    const uint64_t codes = special_codes<R, CC>(P, rl, cl, 0u, 0u, 0u);
-#pragma unroll
-    for (int r = 0; r < R; r++)
-#pragma unroll
-      for (int c = 0; c < CC; c++) {
-        const uint32_t code = (uint32_t)(codes >> (2 * (r * CC + c))) & 3u;
-        if (code == 0u) continue;
-        V[r][c] = code == 1u ? ModelT<MODEL>::NAN_BITS : code == 2u ? 0x7F800000u : 0xFF800000u;
-        dneg0 &= ~(1u << (r * CC + c));
-        to_integer = true;  // the caller rebuilds the integer state from V
-      }
-  }
-}
-
-// switch a thread's state from fp32 values (float-assisted path) to (n, X)
-template <int R, int CC>
-__device__ __forceinline__ void values_to_state(uint32_t (&Np)[R][CC / 2], uint32_t (&V)[R][CC]) {
+  // toward-zero write-back (checked: times 2^896, rounded to nearest, so
+  // that values from 2^128 up become infinite)
 #pragma unroll
   for (int r = 0; r < R; r++)
-#pragma unroll
-    for (int p = 0; p < CC / 2; p++) {
-      int32_t n0, n1, x0, x1;
-      bool z;
-      state_from_fp32(V[r][2 * p], n0, x0, z);
-      state_from_fp32(V[r][2 * p + 1], n1, x1, z);
-      V[r][2 * p] = (uint32_t)x0;
-      V[r][2 * p + 1] = (uint32_t)x1;
-      Np[r][p] = pack16(n0, n1);
-    }
-}
-
-// Packed n and -0 mask of an R x CC block of fp32 values V (raw bits); returns
-// whether all of them suit the float-assisted path (zero, or of magnitude in
-// [2^-FAST_NMAX, 2^FAST_EMAX)).
-template <int R, int CC>
-__device__ __forceinline__ bool classify_values(const uint32_t (&V)[R][CC], uint32_t (&Np)[R][CC / 2],
-                                                uint32_t &dneg0) {
-  dneg0 = 0;
-  bool ok = true;
-#pragma unroll
-  for (int r = 0; r < R; r++) {
-    int32_t n[CC];
 #pragma unroll
     for (int c = 0; c < CC; c++) {
-      const uint32_t field = (V[r][c] >> 23) & 0xFFu;
-      const bool zero = (V[r][c] << 1) == 0u;
-      if (zero && V[r][c]) dneg0 |= 1u << (r * CC + c);
-      n[c] = zero ? ZSENT : 127 - (int32_t)field;
-      ok = ok && (zero || (field >= 127u - FAST_NMAX && field < 127u + FAST_EMAX));
+      constexpr double UP_WB = pow2d(S_WB);
+      const double v = mask24(group_value<F>(X, nm, r, c));
+      X[r][c] = CHK ? __dmul_rn(v, UP_WB) : v;
+    }
+  // signed zeros: only an output whose incoming value was -0 can give -0,
+  // and only when its sum is zero and all its 16 products are zeros of
+  // negative sign
+  if (dneg0) {
+#pragma unroll
+    for (int r = 0; r < R; r++)
+#pragma unroll
+      for (int c = 0; c < CC; c++) {
+        const uint32_t bit = 1u << (r * CC + c);
+        if ((dneg0 & bit) && !(X[r][c] == 0.0 && all_products_negative_zero(&P, rl + r, cl + c))) dneg0 &= ~bit;
+      }
+  }
+  // Inf / NaN operands
+  if (panel_special) {
+    const uint64_t spec = special_codes<R, CC>(&P, rl, cl, c_nan, c_infp, c_infn);
+#pragma unroll
+    for (int r = 0; r < R; r++)
+#pragma unroll
+      for (int c = 0; c < CC; c++) {
+        const uint32_t code = (uint32_t)(spec >> (2 * (r * CC + c))) & 3u;
+        if (code == 0u) continue;
+        X[r][c] = code == 1u ? __longlong_as_double(0x7FF8000000000000ll)
+                             : code == 2u ? __longlong_as_double(0x7FF0000000000000ll)
+                                          : __longlong_as_double((long long)0xFFF0000000000000ull);
+        dneg0 &= ~(1u << (r * CC + c));
+        if (!CHK) to_checked = true;
+      }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// states from C and back to fp32
+// ---------------------------------------------------------------------------
+// The unchecked form takes FP16 / E4M3 blocks whose C values are all +-0 or
+// of magnitude in [2^-126, 2^100): a group with a nonzero product then has
+// e_max >= -28 and a nonzero sum of at least 2^-53, and without one the sum
+// is the carried value itself, so every result stays normal (or zero), and
+// over any K < 2^31 the values stay below 2^101 (FP16 products are below
+// 2^32, E4M3 products below 2^18; truncation never rounds up).
+template <int FMT>
+__device__ __forceinline__ bool unchecked_ok(uint32_t c) {
+  const uint32_t field = (c >> 23) & 0xFFu;
+  return FMT != FMT_BF16 && ((c << 1) == 0u || field - 1u < 226u);
+}
+
+template <int FMT, int R, int CC>
+__device__ __forceinline__ bool init_states(const uint32_t (&cb)[R][CC], double (&X)[R][CC], uint32_t &dneg0) {
+  bool ok = FMT != FMT_BF16;
+  dneg0 = 0;
+#pragma unroll
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int c = 0; c < CC; c++) {
+      ok = ok && unchecked_ok<FMT>(cb[r][c]);
+      if (cb[r][c] == 0x80000000u) dneg0 |= 1u << (r * CC + c);
     }
 #pragma unroll
-    for (int p = 0; p < CC / 2; p++) Np[r][p] = pack16(n[2 * p], n[2 * p + 1]);
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int c = 0; c < CC; c++) {
+      const uint32_t v = cb[r][c];
+      if ((v << 1) == 0u) {
+        X[r][c] = 0.0;
+      } else {
+        const double d = (double)__uint_as_float(v);  // exact; Inf and NaN stay so
+        constexpr double UP_WB = pow2d(S_WB);
+        X[r][c] = (ok || ((v >> 23) & 0xFFu) == 0xFFu) ? d : __dmul_rn(d, UP_WB);
+      }
+    }
+  return !ok;  // checked
+}
+
+template <int MODEL, int R, int CC>
+__device__ __forceinline__ void states_to_fp32(double (&X)[R][CC], bool chk, uint32_t dneg0, uint32_t (&D)[R][CC]) {
+  if (chk) {
+    uint32_t c2[R][CC / 2];
+    carry_codes<true>(X, c2);
+    subnormal_states(X, c2, dneg0);
   }
-  return ok;
+#pragma unroll
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int c = 0; c < CC; c++) {
+      const double x = X[r][c];
+      uint32_t bits;
+      if (x == 0.0) bits = ((dneg0 >> (r * CC + c)) & 1u) ? 0x80000000u : 0u;
+      else if (isnan(x)) bits = ModelT<MODEL>::NAN_BITS;
+      else {
+        constexpr double DOWN_WB = pow2d(-S_WB);
+        bits = __float_as_uint(__double2float_rn(chk ? x * DOWN_WB : x));  // exact (Inf stays Inf)
+      }
+      D[r][c] = bits;
+    }
+}
+
+template <int R, int CC>
+__device__ __forceinline__ void scale_states(double (&X)[R][CC]) {
+#pragma unroll
+  for (int r = 0; r < R; r++)
+#pragma unroll
+    for (int c = 0; c < CC; c++) {
+      constexpr double UP_WB = pow2d(S_WB);
+      X[r][c] = __dmul_rn(X[r][c], UP_WB);
+    }
 }
 
 // raw fp32 bits of an R x CC block (row stride ldc), or +0 if !have_c
@@ -683,83 +535,8 @@ __device__ __forceinline__ void load_bits(const float *C, size_t ldc, bool have_
   }
 }
 
-// fp32 C values of an R x CC block as raw bits with their packed n (the
-// same as load_bits + classify_values, row by row: this order schedules
-// better in the GEMM's prologue)
-template <int R, int CC>
-__device__ __forceinline__ bool load_values(const float *C, size_t ldc, bool have_c, uint32_t (&Np)[R][CC / 2],
-                                            uint32_t (&V)[R][CC], uint32_t &dneg0) {
-  dneg0 = 0;
-  bool ok = true;
-#pragma unroll
-  for (int r = 0; r < R; r++) {
-    if (have_c) {
-#pragma unroll
-      for (int q = 0; q < CC / 4; q++) {
-        const uint4 v = reinterpret_cast<const uint4 *>(C + r * ldc)[q];
-        V[r][4 * q] = v.x; V[r][4 * q + 1] = v.y; V[r][4 * q + 2] = v.z; V[r][4 * q + 3] = v.w;
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < CC; c++) V[r][c] = 0u;
-    }
-    int32_t n[CC];
-#pragma unroll
-    for (int c = 0; c < CC; c++) {
-      const uint32_t field = (V[r][c] >> 23) & 0xFFu;
-      const bool zero = (V[r][c] << 1) == 0u;
-      if (zero && V[r][c]) dneg0 |= 1u << (r * CC + c);
-      n[c] = zero ? ZSENT : 127 - (int32_t)field;
-      ok = ok && (zero || (field >= 127u - FAST_NMAX && field < 127u + FAST_EMAX));
-    }
-#pragma unroll
-    for (int p = 0; p < CC / 2; p++) Np[r][p] = pack16(n[2 * p], n[2 * p + 1]);
-  }
-  return ok;
-}
-
-// state of an R x CC block from fp32 C values (row stride ldc), or +0
-template <int R, int CC>
-__device__ __forceinline__ void load_state(const float *C, size_t ldc, bool have_c, uint32_t (&Np)[R][CC / 2],
-                                           int32_t (&X)[R][CC], uint32_t &dneg0) {
-  dneg0 = 0;
-#pragma unroll
-  for (int r = 0; r < R; r++) {
-    uint32_t cv[CC];
-    if (have_c) {
-#pragma unroll
-      for (int q = 0; q < CC / 4; q++) {
-        const uint4 v = reinterpret_cast<const uint4 *>(C + r * ldc)[q];
-        cv[4 * q] = v.x; cv[4 * q + 1] = v.y; cv[4 * q + 2] = v.z; cv[4 * q + 3] = v.w;
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < CC; c++) cv[c] = 0u;
-    }
-    int32_t n[CC];
-#pragma unroll
-    for (int c = 0; c < CC; c++) {
-      bool nz;
-      state_from_fp32(cv[c], n[c], X[r][c], nz);
-      if (nz) dneg0 |= 1u << (r * CC + c);
-    }
-#pragma unroll
-    for (int p = 0; p < CC / 2; p++) Np[r][p] = pack16(n[2 * p], n[2 * p + 1]);
-  }
-}
-
-template <int R, int CC>
-__device__ __forceinline__ void state_to_fp32(const uint32_t (&Np)[R][CC / 2], const int32_t (&X)[R][CC],
-                                              uint32_t (&D)[R][CC], uint32_t nan_bits) {
-#pragma unroll
-  for (int r = 0; r < R; r++)
-#pragma unroll
-    for (int c = 0; c < CC; c++)
-      D[r][c] = fp32_from_state((c & 1) ? hi16(Np[r][c / 2]) : lo16(Np[r][c / 2]), X[r][c], nan_bits);
-}
-
 // ---------------------------------------------------------------------------
-// raw operand loading and decoding into a panel
+// raw operand loading
 // ---------------------------------------------------------------------------
 template <int FMT>
 struct Raw8 {  // 8 consecutive raw elements
@@ -807,65 +584,48 @@ __device__ __forceinline__ Raw8<FMT> load_col8(const void *base, size_t elem_off
   return r;
 }
 
-// Exact value of a decoded element as a double, m 2^(e - p) with its sign;
-// zero, Inf and NaN become +-2^-500 (the special-value path reads their
-// markers instead).
-template <int FMT>
-__device__ __forceinline__ double dec_value(const Dec &d) {
-  constexpr int P = FmtT<FMT>::P;
-  const double scale = __hiloint2double((1023 - d.n - P) << 20, 0);  // 2^(e - p), normal for every format
-  const double v = d.m ? (double)d.m * scale : 0x1p-500;
-  return d.s ? -v : v;
-}
-
-// Decode 8 k-consecutive elements of A row m (k = 8h .. 8h+7) into a tile
-// kernel's panel (4-column groups, natural order), or of B column n.
-template <int MODEL, int FMT, int BM, int BN>
-__device__ __forceinline__ uint32_t store_a8(Panel<BM, BN> &P, int m, int h, const Raw8<FMT> &raw) {
-  uint32_t special = 0, signs = 0;
+// Decode 8 k-consecutive elements (k = 8h .. 8h+7) of A row m, or of B
+// column n, into a panel; returns the sign-word bits of those 8 elements and
+// whether one of them is Inf or NaN.
+template <int FMT, class PanelT>
+__device__ __forceinline__ uint32_t store_a8(PanelT &P, int m, int h, const Raw8<FMT> &raw, uint32_t &special) {
+  uint32_t bits = 0;
 #pragma unroll
   for (int i = 0; i < 8; i++) {
-    const Dec d = decode<FMT>(raw.get(i));
-    P.aV[8 * h + i][m] = dec_value<FMT>(d);
-    P.aN2[8 * h + i][m] = pack16(d.n, d.n);
-    signs |= (d.s & 1u) << i;
+    const DecElem d = decode_elem<FMT>(raw.get(i));
+    const int k = 8 * h + i;
+    P.aV[k][m] = d.v;
+    P.aQ2[k][m] = d.q | (d.q << 16);
+    bits |= (d.pos << k) | (d.neg << (16 + k));
     special |= d.special;
   }
-  reinterpret_cast<uint8_t *>(&P.aS[m])[h] = (uint8_t)signs;
-  return special;
+  return bits;
 }
-
-template <int FMT, int BM, int BN>
-__device__ __forceinline__ uint32_t store_b8(Panel<BM, BN> &P, int n, int h, const Raw8<FMT> &raw) {
-  uint32_t special = 0, signs = 0;
+template <int FMT, class PanelT>
+__device__ __forceinline__ uint32_t store_b8(PanelT &P, int n, int h, const Raw8<FMT> &raw, uint32_t &special) {
+  uint32_t bits = 0;
 #pragma unroll
   for (int i = 0; i < 8; i++) {
-    const Dec d = decode<FMT>(raw.get(i));
-    P.bV[8 * h + i][n] = dec_value<FMT>(d) * (1.0 + 0x1p-40);  // exact
-    P.bN2[8 * h + i][n] = (int16_t)d.n;
-    signs |= (d.s & 1u) << i;
+    const DecElem d = decode_elem<FMT>(raw.get(i));
+    const int k = 8 * h + i;
+    constexpr double GROW = 1.0 + pow2d(-40);
+    P.bV[k][PanelT::bslot(n)] = d.v * GROW;  // exact
+    P.bQ[k][n] = (int16_t)d.q;
+    bits |= (d.neg << k) | (d.pos << (16 + k));
     special |= d.special;
   }
-  reinterpret_cast<uint8_t *>(&P.bS[n])[h] = (uint8_t)signs;
-  return special;
+  return bits;
 }
 
 // ---------------------------------------------------------------------------
 // GEMM
 // ---------------------------------------------------------------------------
-// Tuning knobs (compile-time): resident blocks per SM and the unroll of the k loops.
-// A block computes GBM x GBN outputs with one warp per 32 x 32 and a 4 x 8
-// block of outputs per thread.  Measured: 64 x 64 blocks of 128 threads, 4
-// per SM, are 3-5% faster than 64 x 128 blocks of 256 threads, 2 per SM (the
-// same registers and warps per SM, but half as many warps wait at each
-// block's per-chunk barrier).
-#ifndef MMAEMU_GBN
-#define MMAEMU_GBN 64
-#endif
+// A block computes 64 x 64 outputs with 128 threads, one warp per 32 x 32
+// and a 4 x 8 block of outputs per thread; MMAEMU_GMINB blocks per SM.
 #ifndef MMAEMU_GMINB
-#define MMAEMU_GMINB (256 / MMAEMU_GBN)
+#define MMAEMU_GMINB 4
 #endif
-constexpr int GBM = 64, GBN = MMAEMU_GBN, GWN = GBN / 32, GTHREADS = 32 * 2 * GWN, GR = 4, GCC = 8;
+constexpr int GBM = 64, GBN = 64, GWN = 2, GTHREADS = 128, GR = 4, GCC = 8;
 using GPanel = Panel<GBM, GBN>;
 
 // Everything a GEMM launch needs.  Element (m, k) of op(A) sits at
@@ -873,7 +633,8 @@ using GPanel = Panel<GBM, GBN>;
 // op(B) at B[k * ldb + n] (tb == 0) or B[n * ldb + k] (tb == 1); C, D and
 // Dref are row-major with their own leading dimensions.  Batch b (blockIdx.z)
 // adds b times the batch stride to every pointer.  D, Dref, fp and mism may
-// each be null; C null means +0.
+// each be null; C null means +0.  The *_n fields are the extents (elements,
+// or bytes for the workspace) the checking build bounds every index by.
 struct GemmParams {
   const void *A, *B;
   const float *C;
@@ -885,92 +646,123 @@ struct GemmParams {
   long long lda, ldb, ldc, ldd, ldr;
   long long sA, sB, sC, sD, sR, sF;
   // decoded operand panels (workspace written by the decode pass): for each
-  // batch entry, 64-row block of A or 128-column block of B, and K chunk, a
-  // blob laid out exactly like that part of a shared-memory panel; and one
-  // special-value flag word per blob
+  // batch entry, 64-row block of A or 64-column block of B, and K chunk, a
+  // blob laid out exactly like that part of a shared-memory panel
   unsigned char *dA, *dB;
-  uint32_t *flags_a, *flags_b;
   int batch;
+  size_t a_n, b_n, c_n, d_n, r_n, fp_n, dA_n, dB_n;
 };
 
-// Decoded panel blobs: the A part (aV, aN2, aS) and the B part (bV, bN2,
-// bS) of a GPanel, stored contiguously in that order.
+// Decoded panel blobs: the A part (aV .. aF) and the B part (bV .. bF) of a
+// GPanel, stored contiguously in that order.
 constexpr size_t ABLOB = offsetof(GPanel, bV), BBLOB = sizeof(GPanel) - offsetof(GPanel, bV);
-constexpr size_t OFF_AN2 = offsetof(GPanel, aN2), OFF_AS = offsetof(GPanel, aS);
-constexpr size_t OFF_BN2 = offsetof(GPanel, bN2) - ABLOB, OFF_BS = offsetof(GPanel, bS) - ABLOB;
-static_assert(ABLOB == 16 * GBM * 8 + 16 * GBM * 4 + GBM * 2 && BBLOB == 16 * GBN * 8 + 16 * GBN * 2 + GBN * 2 &&
+static_assert(ABLOB == 16 * GBM * 8 + 16 * GBM * 4 + GBM * 4 + 16 && BBLOB == 16 * GBN * 8 + 16 * GBN * 2 + GBN * 4 + 16 &&
                   ABLOB % 16 == 0 && BBLOB % 16 == 0,
               "panel layout");
 
-// Decode pass, A side: one thread per 8 k-consecutive elements (row m,
-// chunk j, half h) into the blob of (batch entry, m / 64, j).
-template <int MODEL, int FMT>
-__global__ void __launch_bounds__(256) decode_a_kernel(const GemmParams p) {
+// Decode pass, A side: one block of 128 threads per blob (64 rows x 16 k):
+// thread t decodes k = 8h .. 8h+7 of row m = rb * 64 + (t & 63), h = t >> 6.
+template <int FMT>
+__global__ void __launch_bounds__(128) decode_a_kernel(const GemmParams p) {
   constexpr int ESIZE = FMT == FMT_E4M3 ? 1 : 2;
-  const int nrb = (p.M + GBM - 1) / GBM, nch = p.K / 16;
-  const int m = blockIdx.x * blockDim.x + threadIdx.x;
-  if (m >= nrb * GBM) return;
-  const int j = blockIdx.y >> 1, h = blockIdx.y & 1;
+  __shared__ uint32_t sgn[GBM];
+  const int rb = blockIdx.x, j = blockIdx.y, nrb = gridDim.x, nch = gridDim.y;
   const size_t bz = blockIdx.z;
-  const void *A = static_cast<const unsigned char *>(p.A) + bz * (size_t)p.sA * ESIZE;
+  const int t = threadIdx.x, ml = t & 63, h = t >> 6;
+  const int m = rb * GBM + ml;
+  if (t < GBM) sgn[t] = 0;
+  __syncthreads();
+  bool ok = true;
   const bool valid = m < p.M;
   const size_t k = 16 * (size_t)j + 8 * h, lda = (size_t)p.lda;
-  const Raw8<FMT> raw = !p.ta ? load_row8<FMT>(A, (size_t)m * lda + k, valid) : load_col8<FMT>(A, k * lda + m, lda, valid);
-  const int rb = m / GBM, ml = m % GBM;
-  unsigned char *blob = p.dA + ((bz * nrb + rb) * nch + j) * ABLOB;
-  uint32_t special = 0, signs = 0;
-#pragma unroll
-  for (int i = 0; i < 8; i++) {
-    const Dec d = decode<FMT>(raw.get(i));
-    const size_t kk = (size_t)(8 * h + i);
-    *reinterpret_cast<double *>(blob + (kk * GBM + ml) * 8) = dec_value<FMT>(d);
-    *reinterpret_cast<uint32_t *>(blob + OFF_AN2 + (kk * GBM + ml) * 4) = pack16(d.n, d.n);
-    signs |= (d.s & 1u) << i;
-    special |= d.special;
+  const size_t off = bz * (size_t)p.sA + (!p.ta ? (size_t)m * lda + k : k * lda + m);
+  MMAEMU_CHECK(ok, !valid || (!p.ta ? off + 8 : off + 7 * lda + 1) <= p.a_n);
+  const Raw8<FMT> raw = !p.ta ? load_row8<FMT>(p.A, off, valid && ok) : load_col8<FMT>(p.A, off, lda, valid && ok);
+  const size_t blob_i = (bz * nrb + rb) * (size_t)nch + j;
+  MMAEMU_CHECK(ok, (blob_i + 1) * ABLOB <= p.dA_n);
+  GPanel &P = *reinterpret_cast<GPanel *>(p.dA + blob_i * ABLOB);  // only the A part is written
+  uint32_t special = 0;
+  uint32_t bits = 0;
+  if (ok) bits = store_a8<FMT>(P, ml, h, raw, special);
+  atomicOr(&sgn[ml], bits);
+  const int any = __syncthreads_or((int)special);
+  if (ok && t < GBM) P.aS[t] = sgn[t];
+  if (ok && t == 0) {
+    P.aF[0] = (uint32_t)any;
+    P.aF[1] = P.aF[2] = P.aF[3] = 0;
   }
-  blob[OFF_AS + 2 * ml + h] = (unsigned char)signs;
-  if (special) atomicOr(&p.flags_a[(bz * nrb + rb) * nch + j], 1u);
+  (void)ESIZE;
 }
 
-// Decode pass, B side: one thread per 8 k-consecutive elements of column n.
-template <int MODEL, int FMT>
-__global__ void __launch_bounds__(256) decode_b_kernel(const GemmParams p) {
-  constexpr int ESIZE = FMT == FMT_E4M3 ? 1 : 2;
-  const int ncb = (p.N + GBN - 1) / GBN, nch = p.K / 16;
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= ncb * GBN) return;
-  const int j = blockIdx.y >> 1, h = blockIdx.y & 1;
+// Decode pass, B side: one block of 128 threads per blob (16 k x 64 columns):
+// thread t decodes k = 8h .. 8h+7 of column n = cb * 64 + (t & 63).
+template <int FMT>
+__global__ void __launch_bounds__(128) decode_b_kernel(const GemmParams p) {
+  __shared__ uint32_t sgn[GBN];
+  const int cb = blockIdx.x, j = blockIdx.y, ncb = gridDim.x, nch = gridDim.y;
   const size_t bz = blockIdx.z;
-  const void *B = static_cast<const unsigned char *>(p.B) + bz * (size_t)p.sB * ESIZE;
+  const int t = threadIdx.x, nl = t & 63, h = t >> 6;
+  const int n = cb * GBN + nl;
+  if (t < GBN) sgn[t] = 0;
+  __syncthreads();
+  bool ok = true;
   const bool valid = n < p.N;
   const size_t k = 16 * (size_t)j + 8 * h, ldb = (size_t)p.ldb;
-  const Raw8<FMT> raw = !p.tb ? load_col8<FMT>(B, k * ldb + n, ldb, valid) : load_row8<FMT>(B, (size_t)n * ldb + k, valid);
-  const int cb = n / GBN, nl = n % GBN;
-  unsigned char *blob = p.dB + ((bz * ncb + cb) * nch + j) * BBLOB;
-  uint32_t special = 0, signs = 0;
-#pragma unroll
-  for (int i = 0; i < 8; i++) {
-    const Dec d = decode<FMT>(raw.get(i));
-    const size_t kk = (size_t)(8 * h + i);
-    *reinterpret_cast<double *>(blob + (kk * GBN + bv_slot(nl)) * 8) = dec_value<FMT>(d) * (1.0 + 0x1p-40);  // exact
-    *reinterpret_cast<int16_t *>(blob + OFF_BN2 + (kk * GBN + nl) * 2) = (int16_t)d.n;
-    signs |= (d.s & 1u) << i;
-    special |= d.special;
+  const size_t off = bz * (size_t)p.sB + (!p.tb ? k * ldb + n : (size_t)n * ldb + k);
+  MMAEMU_CHECK(ok, !valid || (!p.tb ? off + 7 * ldb + 1 : off + 8) <= p.b_n);
+  const Raw8<FMT> raw = !p.tb ? load_col8<FMT>(p.B, off, ldb, valid && ok) : load_row8<FMT>(p.B, off, valid && ok);
+  const size_t blob_i = (bz * ncb + cb) * (size_t)nch + j;
+  MMAEMU_CHECK(ok, (blob_i + 1) * BBLOB <= p.dB_n);
+  // the B part of a panel starts ABLOB bytes into it
+  GPanel &P = *reinterpret_cast<GPanel *>(p.dB + blob_i * BBLOB - ABLOB);
+  uint32_t special = 0;
+  uint32_t bits = 0;
+  if (ok) bits = store_b8<FMT>(P, nl, h, raw, special);
+  atomicOr(&sgn[nl], bits);
+  const int any = __syncthreads_or((int)special);
+  if (ok && t < GBN) P.bS[t] = sgn[t];
+  if (ok && t == 0) {
+    P.bF[0] = (uint32_t)any;
+    P.bF[1] = P.bF[2] = P.bF[3] = 0;
   }
-  blob[OFF_BS + 2 * nl + h] = (unsigned char)signs;
-  if (special) atomicOr(&p.flags_b[(bz * ncb + cb) * nch + j], 1u);
 }
 
-// 16-byte asynchronous global -> shared copy
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
-  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+// ---- bulk asynchronous copies completed on an mbarrier --------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// one bulk copy of this GPU's global memory into this block's shared memory
+// (no multicast)
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for a phase with a bound: false when the bound ran out (the caller
+// records a timeout and winds the block down).
+#ifndef MMAEMU_WAIT_LIMIT
+#define MMAEMU_WAIT_LIMIT (1u << 22)
+#endif
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+  for (uint32_t i = 0; i < MMAEMU_WAIT_LIMIT; i++)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
 
 // Blocks are visited in groups of GROUP_ROWS row blocks, column block by
 // column block, so that the blocks resident at one time share A and B
@@ -981,6 +773,7 @@ template <int MODEL, int FMT>
 __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const GemmParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   GPanel *panels = reinterpret_cast<GPanel *>(smem_raw);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + 2 * sizeof(GPanel));
   const int M = p.M, N = p.N, K = p.K;
   const size_t bz = blockIdx.z;
 
@@ -997,114 +790,130 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const Gemm
   const int rl = (warp / GWN) * 32 + (lane >> 2) * GR;
   const int cl = (warp % GWN) * 32 + (lane & 3) * GCC;
   const bool out_valid = (row0 + rl < M) && (col0 + cl < N);
+  bool ok = true;
 
-  // Per chunk, the block copies its decoded A and B blobs (12,416 + 10,368
-  // bytes for 64 x 64 blocks) into the panel with 16-byte asynchronous copies.
+  // Per chunk, thread 0 copies the block's decoded A and B blobs into one of
+  // two panel buffers with two bulk copies completed on that buffer's
+  // mbarrier; the copy of chunk j + 1 overlaps the arithmetic of chunk j.
   const int nchunks = K / 16;
-  const unsigned char *blob_a = p.dA + (bz * nrb + rb) * (size_t)nchunks * ABLOB;
-  const unsigned char *blob_b = p.dB + (bz * ncb + cb) * (size_t)nchunks * BBLOB;
-  const uint32_t *flag_a = p.flags_a + (bz * nrb + rb) * (size_t)nchunks;
-  const uint32_t *flag_b = p.flags_b + (bz * ncb + cb) * (size_t)nchunks;
-  auto issue_chunk = [&](int j, GPanel &P) {
-    const uint4 *sa = reinterpret_cast<const uint4 *>(blob_a + (size_t)j * ABLOB);
-    const uint4 *sb = reinterpret_cast<const uint4 *>(blob_b + (size_t)j * BBLOB);
-    uint4 *da = reinterpret_cast<uint4 *>(&P);
-    uint4 *db = reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(&P) + ABLOB);
-#pragma unroll
-    for (int i = 0; i < (int)((ABLOB / 16 + GTHREADS - 1) / GTHREADS); i++)
-      if (tid + i * GTHREADS < (int)(ABLOB / 16)) cp_async16(da + tid + i * GTHREADS, sa + tid + i * GTHREADS);
-#pragma unroll
-    for (int i = 0; i < (int)((BBLOB / 16 + GTHREADS - 1) / GTHREADS); i++)
-      if (tid + i * GTHREADS < (int)(BBLOB / 16)) cp_async16(db + tid + i * GTHREADS, sb + tid + i * GTHREADS);
-    cp_async_commit();
+  const size_t blob_a0 = (bz * nrb + rb) * (size_t)nchunks, blob_b0 = (bz * ncb + cb) * (size_t)nchunks;
+  MMAEMU_CHECK(ok, (blob_a0 + nchunks) * ABLOB <= p.dA_n && (blob_b0 + nchunks) * BBLOB <= p.dB_n);
+  auto issue_chunk = [&](int j) {
+    GPanel &P = panels[j & 1];
+    mbar_expect_tx(&bars[j & 1], (uint32_t)(ABLOB + BBLOB));
+    bulk_g2s(&P, p.dA + (blob_a0 + j) * ABLOB, (uint32_t)ABLOB, &bars[j & 1]);
+    bulk_g2s(reinterpret_cast<unsigned char *>(&P) + ABLOB, p.dB + (blob_b0 + j) * BBLOB, (uint32_t)BBLOB,
+             &bars[j & 1]);
   };
-  static_assert(ABLOB % 16 == 0 && BBLOB % 16 == 0, "16-byte copies");
-
-  // accumulator: fp32 bits V on the float-assisted path (FP16 / E4M3 while
-  // the values stay in its range), else the integer state (n, X) in V's place
-  uint32_t Np[GR][GCC / 2];
-  uint32_t V[GR][GCC];
-  int32_t(&X)[GR][GCC] = reinterpret_cast<int32_t(&)[GR][GCC]>(V);
-  uint32_t dneg0;
-  const float *Cb = p.C ? p.C + bz * (size_t)p.sC + (size_t)(row0 + rl) * p.ldc + col0 + cl : nullptr;
-  bool fast = load_values<GR, GCC>(Cb, (size_t)p.ldc, Cb != nullptr && out_valid, Np, V, dneg0);
-  if (!kFloatAssisted<FMT>) fast = false;
-  if (!fast) values_to_state<GR, GCC>(Np, V);
-
-  issue_chunk(0, panels[0]);
-  cp_async_wait_all();
+  auto parity = [](int j) { return (uint32_t)(j >> 1) & 1u; };
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    mbar_init_fence();
+  }
   __syncthreads();
-  bool panel_special = (flag_a[0] | flag_b[0]) != 0;
+  if (tid == 0 && ok) issue_chunk(0);
+
+  // states: exact doubles (see mmaemu_core.cuh), from C
+  double X[GR][GCC];
+  uint32_t dneg0;
+  bool chk;
+  {
+    uint32_t cb_[GR][GCC];
+    const size_t c_off = bz * (size_t)p.sC + (size_t)(row0 + rl) * p.ldc + col0 + cl;
+    const bool have_c = p.C != nullptr && out_valid;
+    MMAEMU_CHECK(ok, !have_c || c_off + (GR - 1) * (size_t)p.ldc + GCC <= p.c_n);
+    load_bits<GR, GCC>(p.C + (have_c ? c_off : 0), (size_t)p.ldc, have_c && ok, cb_);
+    chk = init_states<FMT>(cb_, X, dneg0);
+  }
+
+  bool timed_out = false;
+  int abandoned_at = -1;
+#pragma unroll 1
   for (int j = 0; j < nchunks; j++) {
-    bool next_special = false;
-    if (j + 1 < nchunks) {
-      issue_chunk(j + 1, panels[(j + 1) & 1]);
-      next_special = (flag_a[j + 1] | flag_b[j + 1]) != 0;
-    }
-    if constexpr (kFloatAssisted<FMT>) {
-      if (fast) {
-        bool to_integer = false;
-        mma_chunk_fast<MODEL, FMT, GR, GCC>(panels[j & 1], rl, cl, Np, V, dneg0, panel_special, to_integer);
-        if (to_integer) {
-          values_to_state<GR, GCC>(Np, V);
-          fast = false;
-        }
-      } else {
-        mma_chunk<MODEL, FMT, GR, GCC>(panels[j & 1], rl, cl, Np, X, dneg0, panel_special);
-      }
+    if (tid == 0 && ok && j + 1 < nchunks) issue_chunk(j + 1);
+    const GPanel &P = panels[j & 1];
+    if (!mbar_wait_bounded(&bars[j & 1], parity(j))) timed_out = true;
+    const bool panel_special = (P.aF[0] | P.bF[0]) != 0;
+    if constexpr (FMT == FMT_BF16) {
+      bool unused = false;
+      mma_chunk<MODEL, FMT, true>(P, rl, cl, X, dneg0, panel_special, unused);
     } else {
-      mma_chunk<MODEL, FMT, GR, GCC>(panels[j & 1], rl, cl, Np, X, dneg0, panel_special);
+      if (chk) {
+        bool unused = false;
+        mma_chunk<MODEL, FMT, true>(P, rl, cl, X, dneg0, panel_special, unused);
+      } else {
+        bool to_checked = false;
+        mma_chunk<MODEL, FMT, false>(P, rl, cl, X, dneg0, panel_special, to_checked);
+        if (to_checked) {
+          scale_states(X);
+          chk = true;
+        }
+      }
     }
-    if (j + 1 < nchunks) {
-      cp_async_wait_all();
-      __syncthreads();
-      panel_special = next_special;
+    // every thread is done with this buffer before it is refilled (and every
+    // thread learns whether a wait ran out anywhere in the block)
+    if (__syncthreads_or(timed_out)) {
+      abandoned_at = j;
+      break;
     }
+  }
+  if (abandoned_at >= 0) {
+    // a bounded wait ran out: record it and leave the outputs unwritten,
+    // after waiting (bounded) for the copies this block may still have in
+    // flight (chunks up to abandoned_at + 1 were requested)
+    if (tid == 0) {
+      atomicOr(&g_status, STATUS_TIMEOUT);
+      for (int j = abandoned_at; j <= abandoned_at + 1 && j < nchunks; j++)
+        (void)mbar_wait_bounded(&bars[j & 1], parity(j));
+    }
+    return;
   }
 
   // epilogue: store D, compare with the claimed D, per-16x16-tile xorsum
   uint32_t D[GR][GCC];
-  if (fast) {
-#pragma unroll
-    for (int r = 0; r < GR; r++)
-#pragma unroll
-      for (int c = 0; c < GCC; c++) D[r][c] = V[r][c];
-  } else {
-    state_to_fp32<GR, GCC>(Np, X, D, ModelT<MODEL>::NAN_BITS);
-  }
+  states_to_fp32<MODEL>(X, chk, dneg0, D);
   if (p.D != nullptr && out_valid) {
-    float *Db = p.D + bz * (size_t)p.sD + (size_t)(row0 + rl) * p.ldd + col0 + cl;
+    const size_t d_off = bz * (size_t)p.sD + (size_t)(row0 + rl) * p.ldd + col0 + cl;
+    MMAEMU_CHECK(ok, d_off + (GR - 1) * (size_t)p.ldd + GCC <= p.d_n);
+    if (ok) {
+      float *Db = p.D + d_off;
 #pragma unroll
-    for (int i = 0; i < GR; i++) {
-      uint4 *dst = reinterpret_cast<uint4 *>(Db + (size_t)i * p.ldd);
-      dst[0] = make_uint4(D[i][0], D[i][1], D[i][2], D[i][3]);
-      dst[1] = make_uint4(D[i][4], D[i][5], D[i][6], D[i][7]);
+      for (int i = 0; i < GR; i++) {
+        uint4 *dst = reinterpret_cast<uint4 *>(Db + (size_t)i * p.ldd);
+        dst[0] = make_uint4(D[i][0], D[i][1], D[i][2], D[i][3]);
+        dst[1] = make_uint4(D[i][4], D[i][5], D[i][6], D[i][7]);
+      }
     }
   }
   if (p.Dref != nullptr) {
     // bitwise comparison; the smallest mismatching position of the block is
     // found as the smallest in-block offset (row-major order is preserved)
-    uint32_t count = 0, first = 0xFFFFFFFFu;
+    uint32_t count = 0, firstm = 0xFFFFFFFFu;
     if (out_valid) {
-      const float *Rb = p.Dref + bz * (size_t)p.sR + (size_t)(row0 + rl) * p.ldr + col0 + cl;
+      const size_t r_off = bz * (size_t)p.sR + (size_t)(row0 + rl) * p.ldr + col0 + cl;
+      MMAEMU_CHECK(ok, r_off + (GR - 1) * (size_t)p.ldr + GCC <= p.r_n);
+      if (ok) {
+        const float *Rb = p.Dref + r_off;
 #pragma unroll
-      for (int i = 0; i < GR; i++) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(Rb + (size_t)i * p.ldr);
-        const uint4 v0 = src[0], v1 = src[1];
-        const uint32_t got[GCC] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        for (int i = 0; i < GR; i++) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(Rb + (size_t)i * p.ldr);
+          const uint4 v0 = src[0], v1 = src[1];
+          const uint32_t got[GCC] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-        for (int c = GCC - 1; c >= 0; c--)
-          if (got[c] != D[i][c]) {
-            count++;
-            first = min(first, (uint32_t)((rl + i) * GBN + cl + c));
-          }
+          for (int c = GCC - 1; c >= 0; c--)
+            if (got[c] != D[i][c]) {
+              count++;
+              firstm = min(firstm, (uint32_t)((rl + i) * GBN + cl + c));
+            }
+        }
       }
     }
     count = __reduce_add_sync(0xFFFFFFFFu, count);
-    first = __reduce_min_sync(0xFFFFFFFFu, first);
+    firstm = __reduce_min_sync(0xFFFFFFFFu, firstm);
     if (lane == 0 && count != 0) {
       const unsigned long long idx = (unsigned long long)bz * M * N +
-                                     (unsigned long long)(row0 + first / GBN) * N + col0 + first % GBN;
+                                     (unsigned long long)(row0 + firstm / GBN) * N + col0 + firstm % GBN;
       atomicAdd(&p.mism[0], (unsigned long long)count);
       atomicMin(&p.mism[1], idx);
     }
@@ -1121,7 +930,9 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const Gemm
     x ^= __shfl_xor_sync(0xFFFFFFFFu, x, 8);
     if (out_valid && (lane & 0xD) == 0) {
       const int tr = (row0 + rl) >> 4, tc = (col0 + cl) >> 4;
-      p.fp[bz * (size_t)p.sF + (size_t)tr * (N >> 4) + tc] = x;
+      const size_t f_off = bz * (size_t)p.sF + (size_t)tr * (N >> 4) + tc;
+      MMAEMU_CHECK(ok, f_off < p.fp_n);
+      if (ok) p.fp[f_off] = x;
     }
   }
 }
@@ -1149,26 +960,26 @@ __global__ void __launch_bounds__(TWARPS * 32, 3) tiles_kernel(const void *__res
   auto load_a = [&](size_t u) { return load_row8<FMT>(A, u * 256 + lm * 16 + 8 * lh, true); };
   auto load_b = [&](size_t u) { return load_col8<FMT>(B, u * 256 + (8 * lh) * 16 + lm, 16, true); };
   auto load_c = [&](size_t u, uint32_t(&cv)[TR][TCC]) {
-    load_bits<TR, TCC>(C + u * 256 + rl * 16 + cl, 16, C != nullptr, cv);
+    load_bits<TR, TCC>(C + (C != nullptr ? u * 256 + rl * 16 + cl : 0), 16, C != nullptr, cv);
   };
   Raw8<FMT> ra = load_a(t), rb = load_b(t);
   uint32_t cnext[TR][TCC];
   load_c(t, cnext);
-  uint32_t Np[TR][TCC / 2];
-  uint32_t V[TR][TCC];
-  int32_t(&X)[TR][TCC] = reinterpret_cast<int32_t(&)[TR][TCC]>(V);
+  double X[TR][TCC];
   uint32_t dneg0;
   for (;;) {
-#pragma unroll
-    for (int i = 0; i < TR; i++)
-#pragma unroll
-      for (int c = 0; c < TCC; c++) V[i][c] = cnext[i][c];
-    bool fast = classify_values<TR, TCC>(V, Np, dneg0);
-    if (!kFloatAssisted<FMT>) fast = false;
-    if (!fast) values_to_state<TR, TCC>(Np, V);
+    bool chk = init_states<FMT>(cnext, X, dneg0);
     __syncwarp();  // the previous tile's reads of P are done
-    uint32_t sp = store_a8<MODEL, FMT>(P, lm, lh, ra);
-    sp |= store_b8<FMT>(P, lm, lh, rb);
+    uint32_t sp = 0;
+    const uint32_t abits = store_a8<FMT>(P, lm, lh, ra, sp);
+    const uint32_t bbits = store_b8<FMT>(P, lm, lh, rb, sp);
+    // sign words: the two half-rows (half-columns) of a row (column) meet
+    const uint32_t aw = abits | __shfl_xor_sync(0xFFFFFFFFu, abits, 16);
+    const uint32_t bw = bbits | __shfl_xor_sync(0xFFFFFFFFu, bbits, 16);
+    if (lh == 0) {
+      P.aS[lm] = aw;
+      P.bS[lm] = bw;
+    }
     const bool panel_special = __any_sync(0xFFFFFFFFu, sp != 0);
     __syncwarp();
     const size_t next = t + stride;
@@ -1177,27 +988,24 @@ __global__ void __launch_bounds__(TWARPS * 32, 3) tiles_kernel(const void *__res
       rb = load_b(next);
       load_c(next, cnext);
     }
-    uint32_t D[TR][TCC];
-    if constexpr (kFloatAssisted<FMT>) {
-      bool to_integer = false;
-      if (fast) {
-        mma_chunk_fast<MODEL, FMT, TR, TCC>(P, rl, cl, Np, V, dneg0, panel_special, to_integer);
-        if (to_integer) values_to_state<TR, TCC>(Np, V);
-      } else {
-        mma_chunk<MODEL, FMT, TR, TCC>(P, rl, cl, Np, X, dneg0, panel_special);
-      }
-      if (fast && !to_integer) {
-#pragma unroll
-        for (int i = 0; i < TR; i++)
-#pragma unroll
-          for (int c = 0; c < TCC; c++) D[i][c] = V[i][c];
-      } else {
-        state_to_fp32<TR, TCC>(Np, X, D, ModelT<MODEL>::NAN_BITS);
-      }
+    if constexpr (FMT == FMT_BF16) {
+      bool unused = false;
+      mma_chunk<MODEL, FMT, true>(P, rl, cl, X, dneg0, panel_special, unused);
     } else {
-      mma_chunk<MODEL, FMT, TR, TCC>(P, rl, cl, Np, X, dneg0, panel_special);
-      state_to_fp32<TR, TCC>(Np, X, D, ModelT<MODEL>::NAN_BITS);
+      if (chk) {
+        bool unused = false;
+        mma_chunk<MODEL, FMT, true>(P, rl, cl, X, dneg0, panel_special, unused);
+      } else {
+        bool to_checked = false;
+        mma_chunk<MODEL, FMT, false>(P, rl, cl, X, dneg0, panel_special, to_checked);
+        if (to_checked) {
+          scale_states(X);
+          chk = true;
+        }
+      }
     }
+    uint32_t D[TR][TCC];
+    states_to_fp32<MODEL>(X, chk, dneg0, D);
 #pragma unroll
     for (int i = 0; i < TR; i++)
       *reinterpret_cast<uint4 *>(Dout + t * 256 + (rl + i) * 16 + cl) = make_uint4(D[i][0], D[i][1], D[i][2], D[i][3]);
@@ -1226,6 +1034,24 @@ __global__ void __launch_bounds__(256) xorsum_kernel(const uint4 *__restrict__ v
     uint32_t y = 0;
     for (int w = 0; w < (int)(blockDim.x >> 5); w++) y ^= part[w];
     atomicXor(out, y);
+  }
+}
+
+// A kernel whose only job is a bounded wait that nothing completes: thread 0
+// arms an mbarrier for bytes that never arrive and waits on it with a bound of
+// `spins` tries, then records a timeout exactly as the GEMM does.  Used to
+// check that a wait that runs out leaves the device usable and is reported.
+__global__ void __launch_bounds__(32) wait_timeout_kernel(uint32_t spins, uint32_t *out) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_init_fence();
+    mbar_expect_tx(&bar, 16);  // arrives, but 16 transaction bytes stay pending
+    uint32_t i = 0;
+    bool done = false;
+    for (; i < spins && !done; i++) done = mbar_try_wait(&bar, 0);
+    if (!done) atomicOr(&g_status, STATUS_TIMEOUT);
+    *out = done ? 1u : 0u;
   }
 }
 
@@ -1351,11 +1177,13 @@ int check_device(int *sms = nullptr) {
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 // Library-private stream-ordered memory pool per device for the GEMM's
-// decoded-operand workspace.  Freed workspace stays in the pool (release
-// threshold: unlimited) so that repeated GEMMs reuse it without new
-// device allocations; mmaemu_trim_workspace returns it.
+// decoded-operand workspace.  By default its release threshold is 0: memory
+// freed by a GEMM goes back to the device at the next synchronisation, so
+// nothing stays allocated between calls.  mmaemu_set_workspace_cache(1)
+// raises the threshold so that repeated GEMMs reuse the memory instead.
 std::mutex g_pool_mutex;
 cudaMemPool_t g_pool[kMaxDevices] = {};
+bool g_cache[kMaxDevices] = {};
 
 cudaMemPool_t workspace_pool() {
   int dev = 0;
@@ -1368,7 +1196,7 @@ cudaMemPool_t workspace_pool() {
     props.location.id = dev;
     cudaMemPool_t pool = nullptr;
     if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
-    uint64_t threshold = UINT64_MAX;
+    uint64_t threshold = g_cache[dev] ? UINT64_MAX : 0;
     if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &threshold) != cudaSuccess) {
       cudaMemPoolDestroy(pool);
       return nullptr;
@@ -1396,11 +1224,10 @@ bool valid_pair(int model, int fmt) {
     return MMAEMU_EINVAL;                                                               \
   } while (0)
 
-// Workspace sizes of one GEMM (all batch entries): decoded A and B blobs
-// and their flag words.
+// Workspace sizes of one GEMM (all batch entries): decoded A and B blobs.
 struct GemmSizes {
   int nrb, ncb, nch;
-  size_t a_bytes, b_bytes, fa_bytes, fb_bytes;
+  size_t a_bytes, b_bytes;
 };
 GemmSizes gemm_sizes(int M, int N, int K, int batch) {
   GemmSizes z;
@@ -1409,33 +1236,43 @@ GemmSizes gemm_sizes(int M, int N, int K, int batch) {
   z.nch = K / 16;
   z.a_bytes = (size_t)batch * z.nrb * z.nch * mmaemu::ABLOB;
   z.b_bytes = (size_t)batch * z.ncb * z.nch * mmaemu::BBLOB;
-  z.fa_bytes = (size_t)batch * z.nrb * z.nch * sizeof(uint32_t);
-  z.fb_bytes = (size_t)batch * z.ncb * z.nch * sizeof(uint32_t);
   return z;
 }
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Decode pass for B (p.dB, p.flags_b set) on `stream`.
+// Extents (one past the largest element index) of every buffer a GEMM
+// touches, for the checking build's bounds checks.
+void set_extents(mmaemu::GemmParams &p, int batch) {
+  const size_t bm1 = (size_t)(batch - 1);
+  const size_t a_rows = p.ta ? (size_t)p.K : (size_t)p.M, a_row = p.ta ? (size_t)p.M : (size_t)p.K;
+  const size_t b_rows = p.tb ? (size_t)p.N : (size_t)p.K, b_row = p.tb ? (size_t)p.K : (size_t)p.N;
+  p.a_n = bm1 * (size_t)p.sA + (a_rows - 1) * (size_t)p.lda + a_row;
+  p.b_n = bm1 * (size_t)p.sB + (b_rows - 1) * (size_t)p.ldb + b_row;
+  p.c_n = p.C ? bm1 * (size_t)p.sC + (size_t)(p.M - 1) * p.ldc + p.N : 0;
+  p.d_n = p.D ? bm1 * (size_t)p.sD + (size_t)(p.M - 1) * p.ldd + p.N : 0;
+  p.r_n = p.Dref ? bm1 * (size_t)p.sR + (size_t)(p.M - 1) * p.ldr + p.N : 0;
+  p.fp_n = p.fp ? bm1 * (size_t)p.sF + (size_t)(p.M / 16) * (p.N / 16) : 0;
+}
+
+// Decode pass for B (p.dB set) on `stream`.
 template <int MODEL, int FMT>
 int launch_decode_b(const mmaemu::GemmParams &p, int batch, cudaStream_t stream) {
   const GemmSizes z = gemm_sizes(p.M, p.N, p.K, batch);
-  if (cudaMemsetAsync(p.flags_b, 0, z.fb_bytes, stream) != cudaSuccess) return MMAEMU_ECUDA;
-  const dim3 gb((z.ncb * mmaemu::GBN + 255) / 256, 2 * z.nch, batch);
-  mmaemu::decode_b_kernel<MODEL, FMT><<<gb, 256, 0, stream>>>(p);
+  mmaemu::decode_b_kernel<FMT><<<dim3(z.ncb, z.nch, batch), 128, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
 }
+
+constexpr size_t kGemmSmem = 2 * sizeof(mmaemu::GPanel) + 16;  // two panel buffers and their mbarriers
 
 // Decode pass for A and the MMA kernel (B already decoded) on `stream`.
 template <int MODEL, int FMT>
 int launch_decode_a_gemm(const mmaemu::GemmParams &p, int batch, cudaStream_t stream) {
   const GemmSizes z = gemm_sizes(p.M, p.N, p.K, batch);
-  const size_t smem = 2 * sizeof(mmaemu::GPanel);
   auto kern = mmaemu::gemm_kernel<MODEL, FMT>;
-  if (cudaMemsetAsync(p.flags_a, 0, z.fa_bytes, stream) != cudaSuccess ||
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem) != cudaSuccess)
     return MMAEMU_ECUDA;
-  const dim3 ga((z.nrb * mmaemu::GBM + 255) / 256, 2 * z.nch, batch);
-  mmaemu::decode_a_kernel<MODEL, FMT><<<ga, 256, 0, stream>>>(p);
-  kern<<<dim3(z.ncb, z.nrb, batch), mmaemu::GTHREADS, smem, stream>>>(p);
+  mmaemu::decode_a_kernel<FMT><<<dim3(z.nrb, z.nch, batch), 128, 0, stream>>>(p);
+  kern<<<dim3(z.ncb, z.nrb, batch), mmaemu::GTHREADS, kGemmSmem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
 }
 
@@ -1443,18 +1280,18 @@ template <int MODEL, int FMT>
 int launch_gemm(const mmaemu::GemmParams &p_in, int batch) {
   mmaemu::GemmParams p = p_in;
   const GemmSizes z = gemm_sizes(p.M, p.N, p.K, batch);
-  // workspace: decoded blobs and their flags, stream-ordered, released
-  // after the GEMM
+  // workspace: decoded blobs, stream-ordered, released after the GEMM
   unsigned char *ws = nullptr;
   cudaMemPool_t pool = workspace_pool();
-  if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws),
-                                       z.a_bytes + z.b_bytes + z.fa_bytes + z.fb_bytes, pool, t_stream) != cudaSuccess)
+  const size_t total = up256(z.a_bytes) + up256(z.b_bytes);
+  if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), total, pool, t_stream) != cudaSuccess)
     return MMAEMU_ECUDA;
   p.dA = ws;
-  p.dB = ws + z.a_bytes;
-  p.flags_a = reinterpret_cast<uint32_t *>(ws + z.a_bytes + z.b_bytes);
-  p.flags_b = reinterpret_cast<uint32_t *>(ws + z.a_bytes + z.b_bytes + z.fa_bytes);
+  p.dB = ws + up256(z.a_bytes);
+  p.dA_n = z.a_bytes;
+  p.dB_n = z.b_bytes;
   p.batch = batch;
+  set_extents(p, batch);
   int rc = launch_decode_b<MODEL, FMT>(p, batch, t_stream);
   if (rc == MMAEMU_OK) rc = launch_decode_a_gemm<MODEL, FMT>(p, batch, t_stream);
   if (cudaFreeAsync(ws, t_stream) != cudaSuccess) rc = MMAEMU_ECUDA;
@@ -1505,12 +1342,11 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
   const GemmSizes zs = gemm_sizes(rows_per, N, K, 1), zb = gemm_sizes(M, N, K, 1);
   const size_t a_bytes = (size_t)M * K * ES, b_bytes = (size_t)K * N * ES, cd_bytes = (size_t)M * N * 4;
   const size_t fp_bytes = fp_h ? (size_t)(M / 16) * (N / 16) * 4 : 0;
-  // device buffers, each 256-byte aligned inside one pool allocation
-  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  const size_t o_b = up(a_bytes), o_c = o_b + up(b_bytes), o_d = o_c + (C_h ? up(cd_bytes) : 0);
-  // two A-blob workspaces and flag arrays, one per compute stream
-  const size_t o_fp = o_d + up(cd_bytes), o_wa = o_fp + up(fp_bytes), o_wb = o_wa + 2 * up(zs.a_bytes);
-  const size_t o_fa = o_wb + up(zb.b_bytes), o_fb = o_fa + 2 * up(zs.fa_bytes), total = o_fb + up(zb.fb_bytes);
+  // device buffers, each 256-byte aligned inside one pool allocation; two
+  // A-blob workspaces, one per compute stream
+  const size_t o_b = up256(a_bytes), o_c = o_b + up256(b_bytes), o_d = o_c + (C_h ? up256(cd_bytes) : 0);
+  const size_t o_fp = o_d + up256(cd_bytes), o_wa = o_fp + up256(fp_bytes), o_wb = o_wa + 2 * up256(zs.a_bytes);
+  const size_t total = o_wb + up256(zb.b_bytes);
   unsigned char *buf = nullptr;
   cudaMemPool_t pool = workspace_pool();
   if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void **>(&buf), total, pool, t_stream) != cudaSuccess)
@@ -1549,8 +1385,9 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
   }
   mmaemu::GemmParams p = row_major_params(M, N, K, dA, dB, dC, dD, dfp);
   p.dB = buf + o_wb;
-  p.flags_b = reinterpret_cast<uint32_t *>(buf + o_fb);
+  p.dB_n = zb.b_bytes;
   p.batch = 1;
+  set_extents(p, 1);
   if (rc == MMAEMU_OK && ok(cudaStreamWaitEvent(t_stream, e_b, 0))) rc = launch_decode_b<MODEL, FMT>(p, 1, t_stream);
   if (rc == MMAEMU_OK && ok(cudaEventRecord(e_bdec, t_stream))) ok(cudaStreamWaitEvent(c2, e_bdec, 0));
   for (int sl = 0; sl < nslab && rc == MMAEMU_OK; sl++) {
@@ -1563,8 +1400,9 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
     q.C = dC ? dC + r0 * N : nullptr;
     q.D = dD + r0 * N;
     q.fp = dfp ? dfp + (r0 / 16) * (N / 16) : nullptr;
-    q.dA = buf + o_wa + (sl & 1) * up(zs.a_bytes);
-    q.flags_a = reinterpret_cast<uint32_t *>(buf + o_fa + (sl & 1) * up(zs.fa_bytes));
+    q.dA = buf + o_wa + (sl & 1) * up256(zs.a_bytes);
+    q.dA_n = zs.a_bytes;
+    set_extents(q, 1);
     if (!ok(cudaStreamWaitEvent(st, e_in(sl), 0))) break;
     rc = launch_decode_a_gemm<MODEL, FMT>(q, 1, st);
     if (rc != MMAEMU_OK || !ok(cudaEventRecord(e_done(sl), st)) || !ok(cudaStreamWaitEvent(s_out, e_done(sl), 0)))
@@ -1598,8 +1436,8 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
 int validate_gemm(const mmaemu::GemmParams &p, long long batch) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0 || (p.M & 15) || (p.N & 15) || (p.K & 15)) return MMAEMU_EINVAL;
   if (batch < 1 || batch > 65535) return MMAEMU_EINVAL;
-  if ((long long)p.M / mmaemu::GBM >= 65535) return MMAEMU_EINVAL;
-  if ((long long)p.K / 16 * 2 > 65535) return MMAEMU_EINVAL;  // decode-pass grid
+  if ((long long)p.M / mmaemu::GBM >= 65535) return MMAEMU_EINVAL;  // grid y (row blocks)
+  if ((long long)p.K / 8 > 65535) return MMAEMU_EINVAL;             // decode-pass grid y (chunks), with margin
   if (!p.A || !p.B) return MMAEMU_EINVAL;
   if (!p.D && !p.fp && !p.Dref) return MMAEMU_EINVAL;  // nothing to produce
   if (p.Dref && !p.mism) return MMAEMU_EINVAL;
@@ -1641,7 +1479,6 @@ int run_gemm(int model, int fmt, mmaemu::GemmParams &p, long long batch) {
 #undef CALL_GEMM
 }
 
-
 template <int MODEL, int FMT>
 int launch_tiles(const void *A, const void *B, const float *C, float *D, size_t ntiles, int sms) {
   const size_t smem = mmaemu::TWARPS * sizeof(mmaemu::TPanel);
@@ -1658,7 +1495,6 @@ int launch_tiles(const void *A, const void *B, const float *C, float *D, size_t 
   kern<<<blocks, mmaemu::TWARPS * 32, smem, t_stream>>>(A, B, C, D, ntiles);
   return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
 }
-
 
 }  // namespace
 
@@ -1780,6 +1616,35 @@ int mmaemu_xorsum(const void *D, size_t n, uint32_t *out_host) {
   return rc;
 }
 
+int mmaemu_set_workspace_cache(int enable) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MMAEMU_ECUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MMAEMU_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_pool_mutex);
+  g_cache[dev] = enable != 0;
+  if (g_pool[dev]) {
+    uint64_t threshold = enable ? UINT64_MAX : 0;
+    if (cudaMemPoolSetAttribute(g_pool[dev], cudaMemPoolAttrReleaseThreshold, &threshold) != cudaSuccess)
+      return MMAEMU_ECUDA;
+    if (!enable && cudaMemPoolTrimTo(g_pool[dev], 0) != cudaSuccess) return MMAEMU_ECUDA;
+  }
+  return MMAEMU_OK;
+}
+
+int mmaemu_workspace_reserved(size_t *bytes) {
+  if (!bytes) return MMAEMU_EINVAL;
+  *bytes = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MMAEMU_ECUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MMAEMU_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_pool_mutex);
+  if (!g_pool[dev]) return MMAEMU_OK;
+  uint64_t v = 0;
+  if (cudaMemPoolGetAttribute(g_pool[dev], cudaMemPoolAttrReservedMemCurrent, &v) != cudaSuccess) return MMAEMU_ECUDA;
+  *bytes = (size_t)v;
+  return MMAEMU_OK;
+}
+
 int mmaemu_trim_workspace(void) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MMAEMU_ECUDA;
@@ -1789,15 +1654,57 @@ int mmaemu_trim_workspace(void) {
   return MMAEMU_OK;
 }
 
+int mmaemu_device_status(int clear, uint32_t *bits_out) {
+  int rc = check_device();
+  if (rc != MMAEMU_OK) return rc;
+  if (cudaStreamSynchronize(t_stream) != cudaSuccess) return MMAEMU_ECUDA;
+  uint32_t bits = 0;
+  if (cudaMemcpyFromSymbol(&bits, mmaemu::g_status, sizeof bits) != cudaSuccess) return MMAEMU_ECUDA;
+  if (clear && bits) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(mmaemu::g_status, &zero, sizeof zero) != cudaSuccess) return MMAEMU_ECUDA;
+  }
+  if (bits_out) *bits_out = bits;
+  if (bits & mmaemu::STATUS_BOUNDS) return MMAEMU_EBOUNDS;
+  if (bits & mmaemu::STATUS_TIMEOUT) return MMAEMU_ETIMEOUT;
+  return MMAEMU_OK;
+}
+
+int mmaemu_selftest_wait_timeout(unsigned spins, int *completed_out) {
+  int rc = check_device();
+  if (rc != MMAEMU_OK) return rc;
+  uint32_t *flag = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void **>(&flag), sizeof(uint32_t), t_stream) != cudaSuccess) return MMAEMU_ECUDA;
+  mmaemu::wait_timeout_kernel<<<1, 32, 0, t_stream>>>(spins, flag);
+  rc = cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
+  uint32_t done = 0;
+  if (rc == MMAEMU_OK &&
+      cudaMemcpyAsync(&done, flag, sizeof done, cudaMemcpyDeviceToHost, t_stream) != cudaSuccess)
+    rc = MMAEMU_ECUDA;
+  if (cudaFreeAsync(flag, t_stream) != cudaSuccess) rc = MMAEMU_ECUDA;
+  if (cudaStreamSynchronize(t_stream) != cudaSuccess) rc = MMAEMU_ECUDA;
+  if (rc == MMAEMU_OK && completed_out) *completed_out = (int)done;
+  return rc;
+}
+
+int mmaemu_bounds_checking(void) {
+#ifdef MMAEMU_BOUNDS_CHECK
+  return 1;
+#else
+  return 0;
+#endif
+}
+
 const char *mmaemu_strerror(int code) {
   switch (code) {
     case MMAEMU_OK: return "ok";
     case MMAEMU_EINVAL: return "invalid argument (enum, model/format pair, pointer, alignment or size)";
     case MMAEMU_ECUDA: return "CUDA runtime error";
-    case MMAEMU_ETIMEOUT: return "bounded device wait expired";
+    case MMAEMU_ETIMEOUT: return "a bounded device wait gave up";
     case MMAEMU_EUNSUPPORTED: return "unsupported: the current CUDA device is not an sm_100 (B200-class) GPU, "
                                      "or the probe cannot be built for this format";
     case MMAEMU_ECALLBACK: return "the MMA callback of a probe reported an error";
+    case MMAEMU_EBOUNDS: return "a bounds check of the checking build failed (an index left its buffer)";
     default: return "unknown error code";
   }
 }
@@ -1808,13 +1715,14 @@ const char *mmaemu_strerror(int code) {
 // xorsum that allocates nothing
 //
 // For callers that cannot allocate device memory at the moment they need a
-// fingerprint -- for instance a verification step that runs after the device has run out
-// of memory, or inside a process whose device memory is entirely reserved by
-// another allocator -- mmaemu_xorsum_noalloc does the same reduction with a
-// fixed scratch array that lives in the library image instead of a per-call
-// allocation.  Each block of xorsum_partials_kernel folds a fixed span of the
-// input into one word of the array; xorsum_finish_kernel folds those words
-// into the result slot, which is then copied to the host.
+// fingerprint -- for instance a verification step that runs after the device
+// has run out of memory, or inside a process whose device memory is entirely
+// reserved by another allocator -- mmaemu_xorsum_noalloc does the same
+// reduction with a fixed scratch array that lives in the library image
+// instead of a per-call allocation.  Each block of xorsum_partials_kernel
+// folds a fixed span of the input into one word of the array;
+// xorsum_finish_kernel folds those words into the result slot, which is then
+// copied to the host.
 // ===========================================================================
 namespace mmaemu {
 
@@ -1875,7 +1783,9 @@ namespace {
 
 // Device address of the scratch array, looked up once per device (with that
 // device current).  In host code the array's name only stands for the device
-// symbol; it is not an address a kernel may be given.
+// symbol; it is not an address a kernel may be given.  The same first call
+// also loads both kernels onto the device (CUDA loads modules lazily, and
+// loading takes device memory), so that later calls need none.
 std::atomic<uint32_t *> g_noalloc_scratch_ptr[kMaxDevices];
 
 int noalloc_scratch(uint32_t **out) {
@@ -1884,6 +1794,10 @@ int noalloc_scratch(uint32_t **out) {
   if (dev < 0 || dev >= kMaxDevices) return MMAEMU_EUNSUPPORTED;
   uint32_t *p = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
   if (p == nullptr) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, mmaemu::xorsum_partials_kernel) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, mmaemu::xorsum_finish_kernel) != cudaSuccess)
+      return MMAEMU_ECUDA;
     if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), mmaemu::g_noalloc_scratch) != cudaSuccess ||
         p == nullptr)
       return MMAEMU_ECUDA;

@@ -10,27 +10,24 @@
 // extended range, max-exponent threshold -133), and Algorithm 10 (final cast
 // to FP32 overflows to infinity).
 //
-// Integer formulation of one output element and one group:
-//  * every term carries n = -e (negated exponent); zero operands get ZSENT so
-//    they never set the group maximum; e_max = max e  <=>  nmin = min n;
-//  * a product contributes its exact magnitude ma mb 2^(ea+eb-2p) truncated
-//    onto the grid 2^(e_max - F), with its sign, so the group sum S is an
-//    exact two's complement integer in units of that grid (the kernels add
-//    each product with one round-toward-zero fused FP64 multiply-add on an
-//    integer held in a double's mantissa; see group_products in mmaemu.cu);
-//  * because ~x shifted arithmetically equals ~(x shifted logically), a carried
-//    term held in ones' complement (the stage-1 result, or C) is aligned with
-//    one arithmetic shift and turned exact by adding its sign bit:
-//    ~(M >> d) + 1 = -(M >> d).
-//
-// Accumulator state between K chunks: (n, X).  X holds the value's magnitude
-// left-aligned with its leading bit at bit 30, in ones' complement for a
-// negative value.  The fp32 significand is X >> 7 (24 bits; bits below 7 may
-// hold extra low bits that every consumer shifts away, except for the Hopper
-// model whose 25-bit grid would see bit 6, so those states are masked).
-// Zeros have n = ZSENT and X = 0 (+0) or -1 (-0); infinities and NaN are
-// carried as the exponent markers STATE_INF / STATE_NAN, large enough that every
-// other term truncates to zero, so they pass through the ordinary arithmetic.
+// Exact-double formulation of one output element and one accumulation group
+// (see group_step in mmaemu.cu):
+//  * every operand carries an exponent code q = (512 - e) * 16 in 16 bits, so
+//    that a product's code qa + qb is ncode(ea + eb) = (1024 - e) * 16; the
+//    carried term's code is read straight from the top 16 bits of its double;
+//    e_max over the group is the minimum code, found two outputs at a time
+//    with packed 16-bit add-and-min;
+//  * the group is summed in a double acc whose value is (1.5 * 2^52 + L) u on
+//    the grid u = 2^(e_max - F): every double in [2^52 u, 2^53 u) is a
+//    multiple of u, so a round-toward-zero fused multiply-add of a term adds
+//    exactly floor(term / u) -- the truncated magnitude for a positive term,
+//    minus one more than it for a negative one (B is stored times 1 + 2^-40,
+//    so no product sits on the grid).  L starts as the number of negative
+//    terms, which makes every term's contribution its sign-magnitude
+//    truncation;
+//  * the exact group value is acc minus the base 1.5 * 2^52 u, one
+//    subtraction; truncating it to 24 significant bits is a mask of the low
+//    29 mantissa bits: the Ampere hand-over and the fp32 write-back.
 #pragma once
 #include <stdint.h>
 
@@ -39,20 +36,26 @@ namespace mmaemu {
 enum : int { MODEL_AMPERE = 0, MODEL_HOPPER = 1, MODEL_B200 = 2 };
 enum : int { FMT_FP16 = 0, FMT_BF16 = 1, FMT_E4M3 = 2 };
 
-// Negated exponent given to zero operands: larger than any real n sum, so a
-// zero term never sets the group's max exponent; sums of two stay far below
-// 2^15, which keeps packed 16-bit arithmetic exact.
-constexpr int ZSENT = 0x2000;
-// Markers for Inf / NaN operands (read only by the special-value path).
-constexpr int NINF = 0x3000;
-constexpr int NNAN = 0x3001;
-// Accumulator-state markers for an infinite / NaN running value: exponents
-// 300 and 400, beyond any finite term (|e| <= 262), so that the marker term
-// sets the group maximum and every other term truncates to zero.
-constexpr int STATE_INF = -300;
-constexpr int STATE_NAN = -400;
-// Floor on the group max exponent, as a bound on nmin: e_max >= -133.
-constexpr int NFLOOR = 133;
+// ---------------------------------------------------------------------------
+// exponent codes
+// ---------------------------------------------------------------------------
+// ncode(e) = (1024 - e) * 16; an operand carries (512 - e) * 16, so the code
+// of a product is the sum of its operands' codes.  Every code of a nonzero
+// finite term lies in [12320, 20416] (BF16 product exponents -252..254).
+__host__ __device__ constexpr int op_code(int e) { return (512 - e) * 16; }
+__host__ __device__ constexpr int ncode(int e) { return (1024 - e) * 16; }
+// Zero, infinite and NaN operands: large enough that a product with one never
+// sets the group maximum (QZ + the smallest operand code > the floor code),
+// small enough that two of them still fit a signed 16-bit lane.
+constexpr int QZ = 14336, QINF = QZ + 1, QNAN = QZ + 2;
+// The -133 threshold on the group's max exponent (BF16 paragraph), and the
+// exponent an fp32 subnormal carried value takes part in the maximum with.
+constexpr int FLOOR_CODE = ncode(-133);  // 18512
+constexpr int SUBN_CODE = ncode(-126);   // 18400
+// A checked state (see group_step) holds its fp32 value times 2^S_WB, so that
+// values from 2^128 up overflow to infinity in the scaling multiply; the
+// checked Ampere hand-over is carried times 2^S_HO.
+constexpr int S_WB = 896, S_HO = 512;
 
 template <int FMT> struct FmtT;
 template <> struct FmtT<FMT_FP16> {
@@ -71,10 +74,12 @@ template <> struct FmtT<FMT_E4M3> {
 template <int MODEL> struct ModelT;
 template <> struct ModelT<MODEL_AMPERE> {
   static constexpr int F = 23;  // 24-bit internal significand
+  static constexpr int STAGE1 = 8;  // {C, P[1..8]}, then {S1, P[9..16]}
   static constexpr uint32_t NAN_BITS = 0x7FC00000u;
 };
 template <> struct ModelT<MODEL_HOPPER> {
   static constexpr int F = 24;  // 25-bit internal significand
+  static constexpr int STAGE1 = 16;  // one 17-term stage
   static constexpr uint32_t NAN_BITS = 0x7FC00000u;
 };
 // B200's own FP16/BF16 tensor-core MMA, as measured with the target tests:
@@ -82,37 +87,19 @@ template <> struct ModelT<MODEL_HOPPER> {
 // 0x7FFFFFFF.
 template <> struct ModelT<MODEL_B200> {
   static constexpr int F = 25;
+  static constexpr int STAGE1 = 16;
   static constexpr uint32_t NAN_BITS = 0x7FFFFFFFu;
 };
-// At F = 25 sixteen products stay below 2^31 but the carried term can push a
-// group sum to 33 bits: products are summed in 32 bits, the carried term is
-// added in 64.
-template <int MODEL> constexpr bool kWideSum = ModelT<MODEL>::F >= 25;
 
-// The floor can only bind for BF16: fp16/e4m3 terms and fp32 C values are all
-// multiples of 2^-149, so coarsening a grid to 2^-156 (or 2^-157) drops
-// nothing and the result is the same with or without it.
+// The -133 floor can only bind for BF16: fp16/e4m3 terms and fp32 C values
+// are all multiples of 2^-149 and every group with a nonzero term has e_max >=
+// -126, so the floor changes nothing for them; a group with no nonzero term
+// sums to zero on any grid.
 template <int FMT> constexpr bool kNeedsFloor = (FMT == FMT_BF16);
 
 // ---------------------------------------------------------------------------
-// integer helpers with defined behaviour for any shift amount
+// bit helpers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t shr_u32(uint32_t x, uint32_t n) {
-  uint32_t r;
-  asm("shr.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));  // n >= 32 gives 0
-  return r;
-}
-__device__ __forceinline__ int32_t shr_s32(int32_t x, uint32_t n) {
-  int32_t r;
-  asm("shr.s32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));  // n >= 32 gives sign fill
-  return r;
-}
-__device__ __forceinline__ uint32_t shl_u32(uint32_t x, uint32_t n) {
-  uint32_t r;
-  asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));  // n >= 32 gives 0
-  return r;
-}
-// packed signed 16-bit pairs
 __device__ __forceinline__ uint32_t vadd2(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("add.s16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -123,81 +110,51 @@ __device__ __forceinline__ uint32_t vmin2(uint32_t a, uint32_t b) {
   asm("min.s16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
-__device__ __forceinline__ int32_t lo16(uint32_t p) { return (int32_t)(int16_t)(p & 0xFFFFu); }
-__device__ __forceinline__ int32_t hi16(uint32_t p) { return (int32_t)p >> 16; }
-__device__ __forceinline__ uint32_t pack16(int32_t lo, int32_t hi) {
+__device__ __forceinline__ uint32_t vminu2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__host__ __device__ constexpr uint32_t pair16(int lo, int hi) {
   return ((uint32_t)lo & 0xFFFFu) | ((uint32_t)hi << 16);
 }
+__device__ __forceinline__ int32_t lo16(uint32_t p) { return (int32_t)(int16_t)(p & 0xFFFFu); }
+__device__ __forceinline__ int32_t hi16(uint32_t p) { return (int32_t)p >> 16; }
 
 // ---------------------------------------------------------------------------
-// operand decode
+// operand decode (one element)
 // ---------------------------------------------------------------------------
-struct Dec {
-  uint32_t m;        // significand with implicit bit (none for subnormals)
-  int32_t n;         // -e, ZSENT for zero, NINF / NNAN for specials
-  uint32_t s;        // 0 or 0xFFFFFFFF
-  uint32_t special;  // 1 for Inf or NaN
-};
-
 // e = max(field, 1) - bias, m = frac + (field != 0) 2^p: subnormals keep the
 // minimum exponent and no implicit bit (they enter the products unchanged).
+// The value is exact as a double; zero, Inf and NaN operands become a zero of
+// their sign (the special-value path reads their codes).  pos / neg: the
+// operand is nonzero and finite with that sign.
+struct DecElem {
+  double v;
+  uint32_t q;  // op_code(e), or QZ / QINF / QNAN
+  uint32_t pos, neg, special;
+};
+
 template <int FMT>
-__device__ __forceinline__ Dec decode(uint32_t x) {
+__device__ __forceinline__ DecElem decode_elem(uint32_t x) {
   using T = FmtT<FMT>;
   constexpr uint32_t EMASK = (1u << T::EBITS) - 1u, FMASK = (1u << T::P) - 1u;
-  const uint32_t field = (x >> T::P) & EMASK;
-  const uint32_t frac = x & FMASK;
-  Dec d;
-  d.s = ((x >> (T::NBITS - 1)) & 1u) ? 0xFFFFFFFFu : 0u;
-  d.m = frac | (field ? (1u << T::P) : 0u);
+  const uint32_t field = (x >> T::P) & EMASK, frac = x & FMASK;
+  const uint32_t s = (x >> (T::NBITS - 1)) & 1u;
+  const uint32_t m = frac | (field ? (1u << T::P) : 0u);
   const int e = (int)(field ? field : 1u) - T::BIAS;
-  d.n = d.m ? -e : ZSENT;
-  if (T::IEEE) {
-    d.special = field == EMASK;
-    if (d.special) {
-      d.n = frac ? NNAN : NINF;
-      d.m = 0;
-    }
-  } else {
-    d.special = (x & 0x7Fu) == 0x7Fu;
-    if (d.special) {
-      d.n = NNAN;
-      d.m = 0;
-    }
-  }
+  const bool special = T::IEEE ? field == EMASK : (x & 0x7Fu) == 0x7Fu;
+  const bool nan = T::IEEE ? (special && frac != 0) : special;
+  DecElem d;
+  d.special = special;
+  const bool nz = m != 0 && !special;
+  d.q = special ? (nan ? QNAN : QINF) : m ? (uint32_t)op_code(e) : (uint32_t)QZ;
+  // 2^(e - p) is a normal double for every format
+  const double mag = nz ? (double)m * __hiloint2double((1023 + e - T::P) << 20, 0) : 0.0;
+  d.v = s ? -mag : mag;
+  d.pos = nz && !s;
+  d.neg = nz && s;
   return d;
-}
-
-// ---------------------------------------------------------------------------
-// accumulator state <-> fp32
-// ---------------------------------------------------------------------------
-// fp32 bits -> (n, X); negzero is set for -0.
-__device__ __forceinline__ void state_from_fp32(uint32_t c, int32_t &n, int32_t &X, bool &negzero) {
-  const uint32_t field = (c >> 23) & 0xFFu, frac = c & 0x7FFFFFu;
-  const uint32_t s = (uint32_t)((int32_t)c >> 31);
-  negzero = false;
-  if (field == 0xFFu) {
-    n = frac ? STATE_NAN : STATE_INF;
-    X = (int32_t)(0x40000000u ^ (frac ? 0u : s));
-  } else if (field == 0u && frac == 0u) {
-    n = ZSENT;
-    X = (int32_t)s;
-    negzero = s != 0u;
-  } else {
-    const uint32_t m = frac | (field ? 0x800000u : 0u);
-    n = field ? 127 - (int)field : 126;
-    X = (int32_t)((m << 7) ^ s);
-  }
-}
-
-// (n, X) -> fp32 bits; nan_bits is the model's NaN pattern.
-__device__ __forceinline__ uint32_t fp32_from_state(int32_t n, int32_t X, uint32_t nan_bits) {
-  const uint32_t s = (uint32_t)(X >> 31);
-  if (n == ZSENT) return s & 0x80000000u;
-  if (n == STATE_NAN) return nan_bits;
-  if (n == STATE_INF) return (s & 0x80000000u) | 0x7F800000u;
-  const uint32_t m = ((uint32_t)X ^ s) >> 7;  // 24-bit significand (no implicit bit if subnormal)
-  return (s & 0x80000000u) | (((uint32_t)(126 - n) << 23) + m);
 }
 
 }  // namespace mmaemu

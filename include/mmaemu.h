@@ -61,9 +61,10 @@ enum { MMAEMU_FP16 = 0, MMAEMU_BF16 = 1, MMAEMU_E4M3 = 2 };
 #define MMAEMU_OK 0
 #define MMAEMU_EINVAL (-1)       /* bad enum or pair, NULL or misaligned pointer, bad size */
 #define MMAEMU_ECUDA (-2)        /* a CUDA runtime call or launch failed                    */
-#define MMAEMU_ETIMEOUT (-3)     /* a bounded device wait gave up (reserved; no call waits) */
+#define MMAEMU_ETIMEOUT (-3)     /* a bounded device wait gave up (mmaemu_device_status)   */
 #define MMAEMU_EUNSUPPORTED (-4) /* the current device is not an sm_100 GPU                 */
 #define MMAEMU_ECALLBACK (-5)    /* a probe's MMA callback failed (mmaemu_probe.h)           */
+#define MMAEMU_EBOUNDS (-6)      /* checking build: an index left its buffer (mmaemu_device_status) */
 
 /* Select the CUDA stream (a cudaStream_t passed as void*) that the calling
  * host thread's later calls enqueue on; NULL selects the legacy default
@@ -84,14 +85,16 @@ int mmaemu_set_stream(void *cuda_stream);
 int mmaemu_tiles(int model, int fmt, const void *A, const void *B, const float *C, float *D,
                  size_t ntiles);
 
-/* GEMM implementation note (all three GEMM calls): each call first decodes
- * A and B once into panel form, then the MMA kernel copies those panels
- * instead of decoding per output block.  The decoded operands live in a
- * stream-ordered workspace of
- *   batch * K/16 * (ceil(M/64) * 12416 + ceil(N/64) * 10368 + small)
- * bytes (about 375 MB for M = N = K = 4096) taken from a memory pool owned
- * by the library.  Freed workspace stays in that pool for the next call;
- * mmaemu_trim_workspace hands it back to the device.  A failed workspace
+/* GEMM implementation note (all GEMM calls): each call first decodes A and
+ * B once into panel form, then the MMA kernel copies those panels instead of
+ * decoding per output block.  The decoded operands live in a stream-ordered
+ * workspace of
+ *   batch * K/16 * (ceil(M/64) * 12560 + ceil(N/64) * 10512) bytes
+ * (about 379 MB for M = N = K = 4096) taken from a memory pool owned by the
+ * library.  By default the pool hands freed workspace back to the device at
+ * the next synchronisation of the stream, event or device, so the library
+ * holds no device memory between calls; mmaemu_set_workspace_cache(1) makes
+ * it keep the memory for the next call instead.  A failed workspace
  * allocation returns MMAEMU_ECUDA before anything is enqueued.            */
 
 /* Large MatMul composed of 16x16x16 tiles (Obs. 4): D = C + A . B where K is
@@ -196,7 +199,10 @@ int mmaemu_xorsum(const void *D, size_t n, uint32_t *out_host);
  *   Limit: n <= MMAEMU_XORSUM_NOALLOC_MAX_WORDS (2^27 words = 512 MiB);
  *   larger n returns MMAEMU_EINVAL before any device work.
  *   The first call on each device looks up the array's device address (with
- *   that device current); make that first call before any stream capture.
+ *   that device current) and loads this call's two kernels onto the device;
+ *   both need device memory once (CUDA loads code lazily).  So make that
+ *   first call while memory is still available -- at start-up, as a
+ *   warm-up -- and before any stream capture; later calls need none.
  *   All calls share the one array: calls whose work overlaps on the GPU (from
  *   different streams or host threads) race and may return wrong values, so
  *   serialise them.  Nothing in the array needs clearing between calls.
@@ -205,10 +211,43 @@ int mmaemu_xorsum(const void *D, size_t n, uint32_t *out_host);
 #define MMAEMU_XORSUM_NOALLOC_MAX_WORDS ((size_t)1 << 27)
 int mmaemu_xorsum_noalloc(const void *D, size_t n, uint32_t *out_host);
 
+/* Keep (enable != 0) or stop keeping (enable == 0) the GEMM workspace on
+ * the current device between calls (see the GEMM implementation note); off
+ * by default.  Turning it off also hands back what is held.  It only trades
+ * device memory for the cost of a stream-ordered allocation per call.
+ * Errors: MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED.                               */
+int mmaemu_set_workspace_cache(int enable);
+
+/* Bytes of device memory the workspace pool of the current device holds at
+ * this moment (0 before the first GEMM on it).  *bytes must not be NULL.
+ * Errors: MMAEMU_EINVAL, MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED.                */
+int mmaemu_workspace_reserved(size_t *bytes);
+
 /* Return the current device's unused GEMM workspace (see above) to the
  * device.  Workspace still in use by enqueued GEMMs is kept.  Errors:
  * MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED.                                       */
 int mmaemu_trim_workspace(void);
+
+/* The device status word of the current device: bits the kernels set since
+ * it was last cleared.  Bit 0: a bounded wait gave up (a GEMM block whose
+ * panel copy did not arrive within its bound stops, records this and
+ * leaves its outputs unwritten).  Bit 1: in the bounds-checking build
+ * (mmaemu_bounds_checking() == 1) an index fell outside its buffer and the
+ * access was skipped.  SYNCHRONOUS: waits for the selected stream first.
+ * clear != 0 resets the word.  bits_out may be NULL.  Returns MMAEMU_EBOUNDS
+ * if bit 1 is set, else MMAEMU_ETIMEOUT if bit 0 is set, else MMAEMU_OK;
+ * MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED on failure.                            */
+int mmaemu_device_status(int clear, uint32_t *bits_out);
+
+/* Exercises the bounded-wait path: launches one block whose wait can never
+ * complete (nothing arrives) with a bound of `spins` tries, which then
+ * records a timeout in the device status word exactly as a GEMM block
+ * would.  *completed_out (may be NULL) receives whether the wait completed
+ * (it does not).  SYNCHRONOUS.  Errors: MMAEMU_ECUDA, MMAEMU_EUNSUPPORTED. */
+int mmaemu_selftest_wait_timeout(unsigned spins, int *completed_out);
+
+/* 1 for the bounds-checking build of the library, 0 otherwise. */
+int mmaemu_bounds_checking(void);
 
 /* Static message for a return code. */
 const char *mmaemu_strerror(int code);

@@ -43,20 +43,33 @@ def L():
 
 
 def test_header_declares_the_boundary():
-    assert declared_functions() == ["mmaemu_gemm", "mmaemu_gemm_host", "mmaemu_gemm_strided_batched", "mmaemu_gemm_verify",
+    assert declared_functions() == ["mmaemu_bounds_checking", "mmaemu_device_status", "mmaemu_gemm",
+                                    "mmaemu_gemm_host", "mmaemu_gemm_strided_batched", "mmaemu_gemm_verify",
                                     "mmaemu_mma_emulated", "mmaemu_mma_native", "mmaemu_model_describe",
                                     "mmaemu_model_identify", "mmaemu_native_tiles",
                                     "mmaemu_probe_alignment_rounding", "mmaemu_probe_floor", "mmaemu_probe_neutral",
                                     "mmaemu_probe_normalization", "mmaemu_probe_precision", "mmaemu_probe_subnormal",
-                                    "mmaemu_probe_writeback_rounding", "mmaemu_set_stream", "mmaemu_strerror",
-                                    "mmaemu_tiles", "mmaemu_trim_workspace", "mmaemu_xorsum",
-                                    "mmaemu_xorsum_noalloc"]
+                                    "mmaemu_probe_writeback_rounding", "mmaemu_selftest_wait_timeout",
+                                    "mmaemu_set_stream", "mmaemu_set_workspace_cache", "mmaemu_strerror",
+                                    "mmaemu_tiles", "mmaemu_trim_workspace", "mmaemu_workspace_reserved",
+                                    "mmaemu_xorsum", "mmaemu_xorsum_noalloc"]
 
 
 def test_library_exports_every_declared_symbol(L):
     for name in declared_functions():
         assert hasattr(L, name), name
         assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+    assert L.mmaemu_bounds_checking() == 0
+
+
+def test_checking_build_exports_every_declared_symbol(L):
+    from bit_exact_tensor_b200 import _build
+
+    C = ctypes.CDLL(_build.LIB_CHECK)
+    for name in declared_functions():
+        assert hasattr(C, name), name
+    C.mmaemu_bounds_checking.restype = ctypes.c_int
+    assert C.mmaemu_bounds_checking() == 1
 
 
 def test_constants_match_python_binding():
@@ -67,7 +80,7 @@ def test_constants_match_python_binding():
     assert c["MMAEMU_FP16"] == m.FORMATS["fp16"] and c["MMAEMU_BF16"] == m.FORMATS["bf16"]
     assert c["MMAEMU_E4M3"] == m.FORMATS["e4m3"]
     assert (c["MMAEMU_OK"], c["MMAEMU_EINVAL"], c["MMAEMU_ECUDA"], c["MMAEMU_ETIMEOUT"],
-            c["MMAEMU_EUNSUPPORTED"], c["MMAEMU_ECALLBACK"]) == (0, -1, -2, -3, -4, -5)
+            c["MMAEMU_EUNSUPPORTED"], c["MMAEMU_ECALLBACK"], c["MMAEMU_EBOUNDS"]) == (0, -1, -2, -3, -4, -5, -6)
     from bit_exact_tensor_b200 import probe
 
     for code, name in probe.ROUNDING.items():
@@ -75,7 +88,7 @@ def test_constants_match_python_binding():
 
 
 def test_strerror_and_set_stream(L):
-    for code in (0, -1, -2, -3, -4, -5, 7):
+    for code in (0, -1, -2, -3, -4, -5, -6, 7):
         assert L.mmaemu_strerror(code)
     assert L.mmaemu_set_stream(None) == 0
 

@@ -4,15 +4,19 @@ import numpy as np
 import pytest
 
 from bit_exact_tensor_b200 import workloads as wl
-from gpu_util import dev_f32, dev_in, first_mismatch, host_bits
+from gpu_util import dev_f32, dev_in, first_mismatch, guarded, guards_intact, host_bits
 
 pytestmark = pytest.mark.gpu
 
 
 def run_tiles(model, fmt, A, B, C):
+    """The tile batch through the binding, D written into a guarded buffer
+    whose guard words must survive."""
     import bit_exact_tensor_b200 as mmaemu
 
-    D = mmaemu.tiles(model, fmt, dev_in(A), dev_in(B), dev_f32(C) if C is not None else None)
+    dbuf, D = guarded((A.shape[0], 16, 16))
+    mmaemu.tiles(model, fmt, dev_in(A), dev_in(B), dev_f32(C) if C is not None else None, out=D)
+    assert guards_intact(dbuf), "D guard words overwritten"
     return host_bits(D)
 
 

@@ -1,4 +1,4 @@
-"""The allocation-free xorsum gives the same value as mmaemu_xorsum.
+"""The allocation-free xorsum gives the same value as mmaemu_xorsum and the oracle.
 
 mmaemu_xorsum_noalloc exists for callers that cannot allocate device memory
 at the point where they need a fingerprint (a check that runs after the
@@ -6,7 +6,9 @@ device ran out of memory, or a process whose device memory is wholly
 reserved by another allocator).  Its scratch is a fixed array in the library
 image, shared by every call, so two calls in a row must each still give the
 right answer whatever the previous call left there.  Both entry points are
-called through the C ABI.
+called through the C ABI, and the value is also checked against the oracle's
+xorsum of the same words.  Once warmed up on a device, a call takes no device
+memory: the free memory the driver reports is the same before and after.
 """
 
 import ctypes
@@ -42,7 +44,7 @@ def _both(L, t, n):
 
 
 @pytest.mark.parametrize("n", [1, 3, 4, 8191, 8192, 8193, 1_000_003, MAX_WORDS])
-def test_noalloc_equals_xorsum_two_calls_in_a_row(n):
+def test_noalloc_equals_xorsum_two_calls_in_a_row(cref, n):
     import torch
 
     L = _abi()
@@ -52,7 +54,25 @@ def test_noalloc_equals_xorsum_two_calls_in_a_row(n):
         t = torch.from_numpy(w.view(np.int32)).cuda()
         ref, got = _both(L, t, n)
         assert got == ref, (n, call)
+        assert got == cref.xorsum(w), (n, call)
         del t
+
+
+def test_noalloc_takes_no_device_memory_once_warm(cref):
+    import torch
+
+    L = _abi()
+    w = np.arange(1 << 20, dtype=np.uint32) * np.uint32(2654435761)
+    t = torch.from_numpy(w.view(np.int32)).cuda()
+    out = ctypes.c_uint32(0)
+    torch.cuda.synchronize()
+    assert L.mmaemu_xorsum_noalloc(t.data_ptr(), w.size, ctypes.byref(out)) == 0  # warm-up
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert L.mmaemu_xorsum_noalloc(t.data_ptr(), w.size, ctypes.byref(out)) == 0
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert out.value == cref.xorsum(w)
 
 
 def test_noalloc_shrinking_sizes_reuse_the_scratch():

@@ -36,24 +36,20 @@ if ROOT not in sys.path:
 
 M = N = K = 4096
 MACS_PER_STEP = M * N * K
-# algorithmic integer ops per emulated MAC in the integer formulation:
-# exponent add, max, shift amount, significand product, truncating shift,
-# sign, accumulate (the INT32-ALU roofline of the metric)
+# algorithmic integer ops per emulated MAC in the integer formulation of the
+# model (exponent add, max, shift amount, significand product, truncating
+# shift, sign, accumulate): the INT32-ALU roofline the metric names
 OPS_PER_MAC = 7
 METRIC = "emulated MACs/s for 4096^3 FP16-Ampere GEMM; % of INT32-ALU roofline; bit-exact"
 UNIT = "MAC/s"
 # Pages' CPU simulator, same workload: 50.8 s per 4096x4096 FP16-Ampere MatMul
 # (K = 4096) on an Apple M4 Pro -> 68.72e9 / 50.8 MAC/s.  Context, not a target.
 PAGES_MACS_PER_S = MACS_PER_STEP / 50.8
-# ALU issue ceiling: 148 SMs x 4 SMSPs x 32 lanes at the 1965 MHz max SM clock.
-SMS, LANES_PER_SM, MAX_SM_MHZ = 148, 128, 1965.0
-ALU_PEAK_TOPS = SMS * LANES_PER_SM * MAX_SM_MHZ * 1e6 / 1e12
-# The kernels do each product's truncating alignment and signed accumulation
-# in one fused FP64 multiply-add (fma.rz.f64): its per-MAC work is bound by
-# the FP64 pipe, 64 lanes per SM per clock (2 cycles per warp instruction on
-# each of the 4 SMSPs) -> 148 x 64 x 1965 MHz fused multiply-adds per second.
-FP64_LANES_PER_SM = 64
-FP64_PEAK_TFMAS = SMS * FP64_LANES_PER_SM * MAX_SM_MHZ * 1e6 / 1e12
+SMS, MAX_SM_MHZ = 148, 1965.0
+# Nominal unit counts, for context only: the rooflines use the issue rates
+# that libmmaemu_peaks measures on the GPU in the same run (lanes per SM per
+# clock, see --pipe-rates and profiles/pipe_rates_b200.md).
+NOMINAL_FP64_LANES, NOMINAL_INT32_LANES = 64, 128
 H2D_BYTES = M * K * 2 + K * N * 2 + M * N * 4
 D2H_BYTES = M * N * 4 + (M // 16) * (N // 16) * 4
 ALGO_BYTES = H2D_BYTES + D2H_BYTES  # A, B, C read and D, fingerprints written once
@@ -61,15 +57,32 @@ WORKLOAD = "gemm M=N=K=4096, Ampere FP16 model, fp32 C=0 and D, fused per-16x16-
 # DRAM bytes per launch of the GEMM kernel (dram__bytes_read.sum + dram__bytes_write.sum)
 # from one ncu capture (its summary is committed under profiles/), valid only
 # for the kernel sources it was taken on, identified by their hash.
-TRAFFIC_CAPTURE = {"source_sha16": "a4cbd92e96d9188a", "bytes": 1_972_282_368}
+TRAFFIC_CAPTURE = {"source_sha16": "", "bytes": 0}
 KERNEL_SOURCES = ("bit_exact_tensor_b200/csrc/mmaemu.cu", "bit_exact_tensor_b200/csrc/mmaemu_core.cuh",
                   "include/mmaemu.h")
+GOLDEN = os.path.join(ROOT, "tests", "golden", "fullsize_gemm.json")
+# workload name -> record name of the stored oracle digests
+GOLDEN_NAMES = {"gemm-ampere-fp16-4096": ("workloads", "cfg3-ampere-fp16-4096"),
+                "gemm-hopper-bf16-4096": ("workloads", "cfg4-hopper-bf16-4096"),
+                "gemm-hopper-bf16-4096-wide": ("workloads", "cfg4b-hopper-bf16-4096-wide"),
+                "gemm-hopper-e4m3-8192x4096x14336": ("workloads", "cfg5-hopper-e4m3-8192x4096x14336")}
+PEAK_OPS = {"dfma": 0, "dadd": 1, "add_min_s16x2": 2, "lop3": 3, "imad": 4, "iadd": 5, "popc_xor": 6, "prmt": 7,
+            "imnmx": 8, "ffma": 9}
 
 
-HBM_PEAK_GBS = 6557.4  # measured STREAM-style copy bandwidth of a B200, GB/s
+def hbm_peak_gbs():
+    """The driver's measured copy bandwidth (MEASURED_PEAKS.json), else the
+    pool's earlier measurement."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "MEASURED_PEAKS.json hbm_gbs (measured copy)"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback 6.65 TB/s (earlier measurement on this pool)"
 DEFAULT_WORKLOAD = "gemm-ampere-fp16-4096"
 PAIRS = (("ampere", "fp16"), ("ampere", "bf16"), ("hopper", "fp16"), ("hopper", "bf16"), ("hopper", "e4m3"),
          ("b200", "fp16"), ("b200", "bf16"))
+GOLDEN_NAMES.update({"tiles-ampere-fp16-4096": ("tiles", "tiles-ampere-fp16-4096")})
+GOLDEN_NAMES.update({f"tiles-{m}-{f}-100k": ("tiles", f"tiles-{m}-{f}-100k") for m, f in PAIRS})
 E4M3_LAYER = "gemm-hopper-e4m3-8192x4096x14336"
 # variants of the E4M3 layer GEMM: fingerprints only (no D written), verify
 # a claimed D instead of storing it, weights stored [N][K] (B transposed)
@@ -164,6 +177,76 @@ def measured_traffic():
     return TRAFFIC_CAPTURE["bytes"] if kernel_source_sha16() == TRAFFIC_CAPTURE["source_sha16"] else None
 
 
+def measure_rates(ops=("dfma", "iadd"), iters=20000):
+    """Issue rates (lanes per SM per clock) of instruction classes, measured
+    on the current GPU by libmmaemu_peaks (see csrc/peaks.cu)."""
+    import ctypes
+
+    from bit_exact_tensor_b200 import _build
+
+    L = ctypes.CDLL(_build.LIB_PEAKS)
+    L.mmaemu_peak_rate.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_double),
+                                   ctypes.POINTER(ctypes.c_double)]
+    L.mmaemu_peak_rate.restype = ctypes.c_int
+    out = {}
+    for op in ops:
+        lanes, secs = ctypes.c_double(0), ctypes.c_double(0)
+        rc = L.mmaemu_peak_rate(PEAK_OPS[op], iters, ctypes.byref(lanes), ctypes.byref(secs))
+        if rc != 0:
+            raise RuntimeError(f"mmaemu_peak_rate({op}) failed: {rc}")
+        out[op] = lanes.value
+    return out
+
+
+def verify_against_oracle(name, D_host, fp_host):
+    """Compare the timed call's result with the oracle's digests stored in
+    tests/golden/fullsize_gemm.json (written by tests/golden/make_fullsize.py
+    from a run of the oracle on every output element).  Returns the record
+    for the JSON line; raises on any difference."""
+    import hashlib
+
+    import numpy as np
+
+    if name not in GOLDEN_NAMES or not os.path.exists(GOLDEN):
+        return {"verified": None, "against": "no stored oracle digest for this workload"}
+    sec, key = GOLDEN_NAMES[name]
+    with open(GOLDEN) as fh:
+        rec = json.load(fh).get(sec, {}).get(key)
+    if rec is None:
+        return {"verified": None, "against": "no stored oracle digest for this workload"}
+    d = np.ascontiguousarray(D_host.view(np.uint32), dtype="<u4")
+    got_d = hashlib.sha256(d.tobytes()).hexdigest()
+    out = {"against": f"oracle digests, tests/golden/fullsize_gemm.json [{sec}][{key}]",
+           "d_sha256_equal": got_d == rec["d_sha256"]}
+    if fp_host is not None and "fp_sha256" in rec:
+        fp = np.ascontiguousarray(fp_host.view(np.uint32), dtype="<u4")
+        out["fp_sha256_equal"] = hashlib.sha256(fp.tobytes()).hexdigest() == rec["fp_sha256"]
+    out["verified"] = all(v for k, v in out.items() if k.endswith("_equal"))
+    if not out["verified"]:
+        raise RuntimeError(f"{name}: the timed result differs from the oracle's ({out})")
+    return out
+
+
+def run_pipe_rates():
+    """Print the measured issue rates of the instruction classes the kernels
+    use, with the SM clock sampled during the probes."""
+    import torch
+
+    torch.cuda.init()
+    with ClockSampler(0) as cs:
+        rates = measure_rates(tuple(PEAK_OPS), iters=100000)
+    clocks = cs.summary()
+    mhz = clocks.get("sm_mhz") or MAX_SM_MHZ
+    line = {"pipe_rates_lanes_per_sm_clk": {k: round(v, 2) for k, v in rates.items()},
+            "sms": torch.cuda.get_device_properties(0).multi_processor_count, "clocks": clocks,
+            "dfma_peak_t_per_s_at_max_clock": rates["dfma"] * SMS * MAX_SM_MHZ * 1e6 / 1e12,
+            "dfma_peak_t_per_s_at_sampled_clock": rates["dfma"] * SMS * mhz * 1e6 / 1e12,
+            "note": "1 block of 1024 threads per SM, 8 independent chains per thread; "
+                    "add_min_s16x2 counts one packed add-and-min per lane, popc_xor an xor and a popc"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -174,6 +257,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOAD_NAMES),
                     help="which workload to time (default: the headline 4096^3 FP16-Ampere GEMM)")
+    ap.add_argument("--pipe-rates", action="store_true",
+                    help="measure the issue rates of the instruction classes the kernels use, and exit")
     return ap.parse_args()
 
 
@@ -372,6 +457,13 @@ def run_gpu(args):
     C = torch.from_numpy(C_np.view(np.int32)).to(dev)
     stream = torch.cuda.current_stream(dev)
     model, fmt = spec["model"], spec["fmt"]
+    # opt in to keeping the GEMM's decoded-operand workspace between calls
+    # (the library's default hands it back after every call); declared in
+    # the JSON line's config
+    mmaemu.set_workspace_cache(True)
+    # kernels of ours per timed step: decode B, decode A, MMA for a GEMM call;
+    # one tile kernel for a tile batch
+    launches_per_step = 3 if spec["kind"] == "gemm" else 1
     if spec["kind"] == "gemm":
         D = torch.empty(C.shape, dtype=torch.float32, device=dev)
         fp = torch.empty(((C.shape[-2] // 16) * (C.shape[-1] // 16),), dtype=torch.int32, device=dev)
@@ -437,6 +529,28 @@ def run_gpu(args):
         count, first = mism.cpu().tolist()
         if count != 0:
             raise RuntimeError(f"verify mode found {count} mismatches (first at {first}) in its own result")
+        verified = {"verified": True, "against": "the call's own claimed D (verify mode), 0 mismatches"}
+    elif mode in ("store", "wt", None) or spec["kind"] == "tiles":
+        # the last timed call's result against the oracle's stored digests
+        base = args.workload[:-3] if mode == "wt" else args.workload  # B stored [N][K]: the same GEMM
+        verified = verify_against_oracle(base, D.cpu().numpy(), fp.cpu().numpy() if spec["kind"] == "gemm" else None)
+    elif mode == "fponly":
+        verified = {"verified": None, "against": "no stored oracle digest for this workload"}
+        if GOLDEN_NAMES.get(args.workload.rsplit("-fponly", 1)[0]):
+            import hashlib
+
+            sec, key = GOLDEN_NAMES[args.workload.rsplit("-fponly", 1)[0]]
+            with open(GOLDEN) as fh:
+                want = json.load(fh)[sec][key]["fp_sha256"]
+            got = hashlib.sha256(np.ascontiguousarray(fp.cpu().numpy().view(np.uint32), dtype="<u4").tobytes())
+            verified = {"verified": got.hexdigest() == want, "against": f"oracle fingerprint digest [{sec}][{key}]"}
+            if not verified["verified"]:
+                raise RuntimeError("fingerprints differ from the oracle's")
+    else:
+        verified = {"verified": None, "against": "no stored oracle digest for this workload"}
+    # issue rates of the FP64 pipe and of the fastest INT32 instruction,
+    # measured now on this GPU (lanes per SM per clock)
+    rates = measure_rates(("dfma", "iadd"))
 
     # end to end through the public API from pinned host buffers
     A_h = torch.from_numpy(A_np.view(in_view)).pin_memory()
@@ -491,38 +605,54 @@ def run_gpu(args):
         macs = spec["macs"]
         value = aggregate_value(total_ms / args.steps, world, macs)
         h2d, d2h = spec["h2d"], spec["d2h"]
-        int_ops = OPS_PER_MAC * macs / (kern_ms / 1e3) / 1e12
-        # one fused FP64 multiply-add per emulated MAC
+        mhz = clocks.get("sm_mhz") or MAX_SM_MHZ
+        # one round-toward-zero FP64 fused multiply-add per emulated MAC: the
+        # bound is the FP64 pipe, at its measured issue rate and the SM clock
+        # sampled during the timed region
+        fp64_peak = rates["dfma"] * SMS * mhz * 1e6 / 1e12
         achieved = macs / (kern_ms / 1e3) / 1e12
-        kernel = (f"gemm_kernel<{spec['model']},{spec['fmt']}> with its decode pass (one call, timed whole)"
+        kernel = (f"gemm_kernel<{spec['model']},{spec['fmt']}> with its two decode kernels (one call, timed whole; "
+                  "the MMA kernel is about 99% of it, profiles/gemm_ampere_fp16_4096_launches.md)"
                   if spec["kind"] == "gemm" else f"tiles_kernel<{spec['model']},{spec['fmt']}>")
-        roof = {"bound": "alu", "achieved": achieved, "peak": FP64_PEAK_TFMAS, "unit": "T FMA/s",
-                "frac": achieved / FP64_PEAK_TFMAS, "kernel": kernel,
-                "fma_per_mac": 1, "peak_basis": "148 SM x 64 FP64 lanes x 1965 MHz (derived)",
-                # the metric's INT32-ALU roofline: the integer formulation's
-                # 7 ops per MAC against the INT32 issue ceiling
-                "int32_alu_frac": int_ops / ALU_PEAK_TOPS, "int32_alu_peak_tops": ALU_PEAK_TOPS,
-                "ops_per_mac_integer_form": OPS_PER_MAC}
+        roof = {"bound": "fp64", "achieved": achieved, "peak": fp64_peak, "unit": "T FMA/s",
+                "frac": achieved / fp64_peak, "kernel": kernel, "fma_per_mac": 1,
+                "peak_basis": (f"DFMA issue rate measured in this run: {rates['dfma']:.1f} lanes/SM/clk "
+                               f"(libmmaemu_peaks; profiles/pipe_rates_b200.md) x {SMS} SMs x {mhz:.0f} MHz "
+                               f"(median SM clock sampled while timing); nominal 64 lanes/SM/clk"),
+                # the metric's INT32-ALU roofline: what the integer formulation
+                # of the model would need (7 integer ops per MAC) against the
+                # measured INT32 issue rate of the fastest integer instruction;
+                # the kernels run one FP64 FMA per MAC instead, so this is an
+                # equivalent, not what binds them
+                "int32_equiv": {"ops_per_mac_integer_form": OPS_PER_MAC,
+                                "peak_tops": rates["iadd"] * SMS * mhz * 1e6 / 1e12,
+                                "peak_basis": f"IADD issue rate measured in this run: {rates['iadd']:.1f} lanes/SM/clk",
+                                "frac": OPS_PER_MAC * achieved / (rates["iadd"] * SMS * mhz * 1e6 / 1e12)}}
         roof.update({"traffic": measured_traffic() if args.workload == DEFAULT_WORKLOAD else None,
                      "traffic_unit": "bytes per launch", "algorithmic_bytes": h2d + d2h})
         if spec["kind"] == "tiles":  # mixed bound: also report HBM against the measured copy bandwidth
             hbm = (h2d + d2h) / (kern_ms / 1e3) / 1e9
-            roof.update({"hbm_achieved_gbs": hbm, "hbm_peak_gbs": HBM_PEAK_GBS, "hbm_frac": hbm / HBM_PEAK_GBS})
+            hbm_peak, hbm_basis = hbm_peak_gbs()
+            roof.update({"hbm_achieved_gbs": hbm, "hbm_peak_gbs": hbm_peak, "hbm_frac": hbm / hbm_peak,
+                         "hbm_peak_basis": hbm_basis})
         line = {
             "metric": METRIC if args.workload == DEFAULT_WORKLOAD else f"emulated MACs/s, {spec['desc']}",
             "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": value / PAGES_MACS_PER_S if args.workload == DEFAULT_WORKLOAD else None,
-            "dtype": "int32", "data": "synthetic",
+            "dtype": "f64", "data": "synthetic",
             "config": {"workload": spec["desc"], "name": args.workload, "emulated_arch": spec["model"],
                        "input_format": spec["fmt"], "global_batch": world,
-                       "parallelism": f"independent x{world}", "l2": spec["l2"]},
+                       "parallelism": f"independent x{world}", "l2": spec["l2"],
+                       "workspace_cache": "on: mmaemu_set_workspace_cache(1) keeps the decoded-operand "
+                                          "workspace between calls (the library default releases it)"},
+            "verified": verified,
             "roofline": roof,
             "clocks": clocks,
             "e2e": {"value": macs * world / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps,
+            "gpu_launches": launches_per_step * args.steps,
         }
         if world == 1 and not args.no_cpu_baseline and args.workload == DEFAULT_WORKLOAD:
             line["cpu_baseline"] = cpu_baseline(inputs=(A_np, B_np, C_np))
@@ -535,6 +665,8 @@ def run_gpu(args):
 
 def main():
     args = parse()
+    if args.pipe_rates:
+        return run_pipe_rates()
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

@@ -5,6 +5,8 @@ libmmaemu_check.so  -- the same sources with MMAEMU_BOUNDS_CHECK: every
                        kernel index is checked against its buffer and a
                        violation is recorded in the device status word
                        instead of being made (selected with MMAEMU_LIB=check).
+libmmaemu_peaks.so  -- issue-rate probes of the instruction classes the
+                       kernels use (bench.py --pipe-rates), for their rooflines.
 """
 
 from __future__ import annotations
@@ -21,6 +23,8 @@ DEPS = SOURCES + [os.path.join(PKG, "csrc", "mmaemu_core.cuh"), os.path.join(ROO
                   os.path.join(ROOT, "include", "mmaemu_probe.h"), os.path.abspath(__file__)]
 LIB = os.path.join(PKG, "libmmaemu.so")
 LIB_CHECK = os.path.join(PKG, "libmmaemu_check.so")
+LIB_PEAKS = os.path.join(PKG, "libmmaemu_peaks.so")
+PEAKS_SRC = os.path.join(PKG, "csrc", "peaks.cu")
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2"]
@@ -43,7 +47,8 @@ def needs_build(lib: str) -> bool:
 
 def _build_one(lib: str, extra: list[str], verbose: bool) -> str:
     tmp = lib + f".{os.getpid()}.tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), *SOURCES, "-o", tmp]
+    srcs = [PEAKS_SRC] if lib == LIB_PEAKS else SOURCES
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"), *srcs, "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
@@ -54,6 +59,8 @@ def _build_one(lib: str, extra: list[str], verbose: bool) -> str:
 def build_library(force: bool = False, verbose: bool = False, checking: bool = True) -> str:
     todo = [(lib, extra) for lib, extra in VARIANTS.items()
             if (checking or lib == LIB) and (force or needs_build(lib))]
+    if force or not os.path.exists(LIB_PEAKS) or os.path.getmtime(LIB_PEAKS) < os.path.getmtime(PEAKS_SRC):
+        todo.append((LIB_PEAKS, []))
     with ThreadPoolExecutor(max_workers=len(todo) or 1) as ex:
         for f in [ex.submit(_build_one, lib, extra, verbose) for lib, extra in todo]:
             f.result()

@@ -115,6 +115,11 @@ __device__ __forceinline__ uint32_t vminu2(uint32_t a, uint32_t b) {
   asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
+__device__ __forceinline__ uint32_t vmaxu2_16(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
 __host__ __device__ constexpr uint32_t pair16(int lo, int hi) {
   return ((uint32_t)lo & 0xFFFFu) | ((uint32_t)hi << 16);
 }

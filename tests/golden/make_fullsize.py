@@ -23,6 +23,7 @@ the CUDA library.  The oracle's wall time for each full workload is stored
 beside the digests (``oracle_seconds``, ``oracle_threads``).
 
   python tests/golden/make_fullsize.py [--only NAME ...] [--threads T]
+  python tests/golden/make_fullsize.py --tiles     # digests of the tile workloads
   python tests/golden/make_fullsize.py --time-only NAME --threads 1
   python tests/golden/make_fullsize.py --time-python-tiles  # Python oracle, 4,096 tiles
 """
@@ -36,6 +37,8 @@ import os
 import platform
 import sys
 import time
+
+import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(os.path.dirname(HERE))
@@ -111,6 +114,36 @@ def host_info() -> dict:
     return {"cpu": cpu, "logical_cpus_available": len(os.sched_getaffinity(0))}
 
 
+def tile_workloads():
+    """The pages' random-tile experiments: 4,096 Ampere-FP16 tiles with
+    subnormals, and 100,000 random + adversarial tiles per model/format
+    pair."""
+    from bit_exact_tensor_b200 import workloads as wl
+
+    out = {"tiles-ampere-fp16-4096": ("ampere", "fp16", wl.config1)}
+    for model, fmt in wl.PAIRS:
+        out[f"tiles-{model}-{fmt}-100k"] = (model, fmt, lambda fmt=fmt: wl.config2(fmt)[:3])
+    return out
+
+
+def run_tiles(threads: int) -> dict:
+    """SHA-256 of the oracle's D for every tile workload."""
+    from oracle import cref
+
+    recs = {}
+    for name, (model, fmt, make) in tile_workloads().items():
+        A, B, C = make()
+        t0 = time.perf_counter()
+        D = cref.tiles(model, fmt, A, B, C, nthreads=threads)
+        dt = time.perf_counter() - t0
+        D = np.ascontiguousarray(D, dtype="<u4")
+        recs[name] = {"model": model, "fmt": fmt, "ntiles": int(A.shape[0]),
+                      "d_sha256": hashlib.sha256(D.tobytes()).hexdigest(),
+                      "specials": special_counts(D), "oracle_seconds": round(dt, 2), "oracle_threads": threads}
+        print(name, recs[name]["oracle_seconds"], "s", flush=True)
+    return recs
+
+
 def time_python_tiles() -> dict:
     """Wall time of the Python oracle (arbitrary-precision integers, one
     element at a time) on the 4,096 Ampere-FP16 tiles of the small tile
@@ -136,6 +169,7 @@ def main() -> int:
     ap.add_argument("--threads", type=int, default=cref.default_threads())
     ap.add_argument("--time-only", default=None, help="time one workload, store only its timing")
     ap.add_argument("--time-python-tiles", action="store_true")
+    ap.add_argument("--tiles", action="store_true", help="store the tile workloads' digests")
     args = ap.parse_args()
 
     data = {}
@@ -144,7 +178,10 @@ def main() -> int:
             data = json.load(fh)
     data.setdefault("workloads", {})
     data.setdefault("timings", {})
-    if args.time_python_tiles:
+    data.setdefault("tiles", {})
+    if args.tiles:
+        data["tiles"].update(run_tiles(args.threads))
+    elif args.time_python_tiles:
         data["timings"]["python_oracle_tiles_4096"] = dict(time_python_tiles(), host=host_info())
     elif args.time_only:
         rec = run_one(args.time_only, args.threads)

@@ -76,10 +76,13 @@ static uint32_t vmin2(uint32_t a, uint32_t b) {
 static uint32_t pair16(int lo, int hi) { return ((uint32_t)lo & 0xFFFFu) | ((uint32_t)hi << 16); }
 
 /* decoded operand: exact value (Inf/NaN/zero as a signed zero), code, sign
- * pair.  A row's sign word has bit k set for a positive nonzero finite a[k]
- * and bit 16+k for a negative one; a B column's word has bit k for a negative
- * b[k] and bit 16+k for a positive one, so that the AND of the two words has
- * one bit per negative product of nonzero finite operands. */
+ * pair.  Sign words: element k = 8h + 2j + b of a row of A (column of B) owns
+ * bit NB(k) = 2j + h + 16b and bit NB(k) + 8.  A row sets NB(k) + 8 for a
+ * positive nonzero finite a[k] and NB(k) for a negative one; a B column sets
+ * NB(k) for a positive b[k] and NB(k) + 8 for a negative one -- so that the
+ * AND of the two words has one bit per negative product of nonzero finite
+ * operands.  k < 8 uses the even bits, k >= 8 the odd ones. */
+static int NB(int k) { return (k & 6) + (k >> 3) + 16 * (k & 1); }
 typedef struct { double v; int q; int pos, neg; int neg_sign; } kdec;
 
 static kdec kdecode(int fmt, uint32_t x) {
@@ -116,12 +119,12 @@ typedef struct {
 
 static uint32_t sign_word_a(const kdec *a) {
   uint32_t w = 0;
-  for (int k = 0; k < 16; k++) w |= ((uint32_t)a[k].pos << k) | ((uint32_t)a[k].neg << (16 + k));
+  for (int k = 0; k < 16; k++) w |= ((uint32_t)a[k].pos << (NB(k) + 8)) | ((uint32_t)a[k].neg << NB(k));
   return w;
 }
 static uint32_t sign_word_b(const kdec *b) {
   uint32_t w = 0;
-  for (int k = 0; k < 16; k++) w |= ((uint32_t)b[k].neg << k) | ((uint32_t)b[k].pos << (16 + k));
+  for (int k = 0; k < 16; k++) w |= ((uint32_t)b[k].pos << NB(k)) | ((uint32_t)b[k].neg << (NB(k) + 8));
   return w;
 }
 
@@ -150,7 +153,7 @@ static void group_pair(const kctx *c, int k0, int kn, const double carry[2], int
   const uint32_t KHI = ((uint32_t)(2099 - c->F) << 20) | 0x80000u;
   const uint32_t hi[2] = {KHI + nm * 0xFFFF0000u, KHI - nm};
   uint32_t gm = 0;
-  for (int k = k0; k < k0 + kn; k++) gm |= 0x10001u << k;
+  for (int k = k0; k < k0 + kn; k++) gm |= 0x101u << NB(k);
   const uint32_t sa = sign_word_a(c->a), sb[2] = {sign_word_b(c->b0), sign_word_b(c->b1)};
 #ifdef MISTAKE_NO_SKEW
   const double growth = 1.0;

@@ -67,7 +67,10 @@ GOLDEN_NAMES = {"gemm-ampere-fp16-4096": ("workloads", "cfg3-ampere-fp16-4096"),
                 "gemm-hopper-bf16-4096-wide": ("workloads", "cfg4b-hopper-bf16-4096-wide"),
                 "gemm-hopper-e4m3-8192x4096x14336": ("workloads", "cfg5-hopper-e4m3-8192x4096x14336")}
 PEAK_OPS = {"dfma": 0, "dadd": 1, "add_min_s16x2": 2, "lop3": 3, "imad": 4, "iadd": 5, "popc_xor": 6, "prmt": 7,
-            "imnmx": 8, "ffma": 9}
+            "imnmx": 8, "ffma": 9,
+            # pairs on independent chains (rate in pairs): do two pipes work at the same time?
+            "pair_dfma_lop3": 10, "pair_dfma_imad": 11, "pair_dfma_ffma": 12, "pair_dfma_add_min_s16x2": 13,
+            "pair_lop3_imad": 14, "pair_lop3_ffma": 15}
 
 
 def hbm_peak_gbs():
@@ -242,7 +245,8 @@ def run_pipe_rates():
             "dfma_peak_t_per_s_at_max_clock": rates["dfma"] * SMS * MAX_SM_MHZ * 1e6 / 1e12,
             "dfma_peak_t_per_s_at_sampled_clock": rates["dfma"] * SMS * mhz * 1e6 / 1e12,
             "note": "1 block of 1024 threads per SM, 8 independent chains per thread; "
-                    "add_min_s16x2 counts one packed add-and-min per lane, popc_xor an xor and a popc"}
+                    "add_min_s16x2 counts one packed add-and-min per lane, popc_xor an xor and a popc; "
+                    "pair_* run both kinds on separate chains and count pairs"}
     print(json.dumps(line), flush=True)
     return 0
 

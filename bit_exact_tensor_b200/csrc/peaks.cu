@@ -9,7 +9,8 @@
 //   int mmaemu_peak_rate(int op, int iters, double *lanes_per_sm_clk,
 //                        double *seconds);
 //     op: one of the PEAK_* codes below; iters: loop iterations per thread
-//     (each runs NCHAIN instructions); one block of 1024 threads per SM.
+//     (each runs NCHAIN instructions, or NCHAIN pairs for the paired codes,
+//     whose rate counts pairs); one block of 1024 threads per SM.
 //     Synchronous; returns 0, or -2 on a CUDA error, -1 on a bad op.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -27,7 +28,14 @@ enum : int {
   PEAK_PRMT = 7,    // prmt.b32
   PEAK_IMNMX = 8,   // min.s32
   PEAK_FFMA = 9,    // fma.rn.f32
-  PEAK_COUNT = 10
+  // pairs of instructions on independent chains: whether two pipes overlap
+  PEAK_DFMA_LOP3 = 10,
+  PEAK_DFMA_IMAD = 11,
+  PEAK_DFMA_FFMA = 12,
+  PEAK_DFMA_ADDMIN2 = 13,
+  PEAK_LOP3_IMAD = 14,
+  PEAK_LOP3_FFMA = 15,
+  PEAK_COUNT = 16
 };
 constexpr int NCHAIN = 8, THREADS = 1024;
 
@@ -60,38 +68,50 @@ __device__ __forceinline__ void step(uint32_t (&u)[NCHAIN], double (&d)[NCHAIN],
   }
 }
 
-template <int OP>
+// Chains of two kinds of instruction (OP2 < 0: one kind) in separate
+// registers; with two kinds each iteration runs NCHAIN of each and the rate
+// counts pairs: the slower kind's rate when the two pipes work at the same
+// time, the harmonic combination when they take turns.
+template <int OP1, int OP2>
 __global__ void __launch_bounds__(THREADS, 1) rate_kernel(int iters, unsigned long long *cycles, uint32_t *sink) {
-  uint32_t u[NCHAIN];
-  double d[NCHAIN];
-  float f[NCHAIN];
+  uint32_t u[NCHAIN], u2[NCHAIN];
+  double d[NCHAIN], d2[NCHAIN];
+  float f[NCHAIN], f2[NCHAIN];
   const uint32_t k = threadIdx.x * 2654435761u + blockIdx.x;
 #pragma unroll
   for (int i = 0; i < NCHAIN; i++) {
     u[i] = k ^ (0x1234567u * (i + 1));
+    u2[i] = u[i] ^ 0x5A5A5A5Au;
     d[i] = 1.0 + i;
+    d2[i] = 2.0 + i;
     f[i] = 1.0f + i;
+    f2[i] = 2.0f + i;
   }
   __syncthreads();
   const unsigned long long t0 = clock64();
 #pragma unroll 1
-  for (int it = 0; it < iters; it++) step<OP>(u, d, f, k + (uint32_t)it);
+  for (int it = 0; it < iters; it++) {
+    step<OP1>(u, d, f, k + (uint32_t)it);
+    if constexpr (OP2 >= 0) step<OP2>(u2, d2, f2, k + (uint32_t)it);
+  }
   __syncthreads();
   const unsigned long long t1 = clock64();
   uint32_t x = 0;
 #pragma unroll
-  for (int i = 0; i < NCHAIN; i++) x ^= u[i] ^ (uint32_t)__double2loint(d[i]) ^ __float_as_uint(f[i]);
+  for (int i = 0; i < NCHAIN; i++)
+    x ^= u[i] ^ u2[i] ^ (uint32_t)__double2loint(d[i]) ^ (uint32_t)__double2loint(d2[i]) ^ __float_as_uint(f[i]) ^
+         __float_as_uint(f2[i]);
   if (x == 0x12345678u) sink[threadIdx.x] = x;  // keeps the chains alive
   if (threadIdx.x == 0) cycles[blockIdx.x] = t1 - t0;
 }
 
-template <int OP>
+template <int OP1, int OP2 = -1>
 int run(int iters, int sms, unsigned long long *cyc, uint32_t *sink, float *ms) {
   cudaEvent_t e0, e1;
   if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) return -2;
-  rate_kernel<OP><<<sms, THREADS>>>(8, cyc, sink);  // warm-up
+  rate_kernel<OP1, OP2><<<sms, THREADS>>>(8, cyc, sink);  // warm-up
   cudaEventRecord(e0);
-  rate_kernel<OP><<<sms, THREADS>>>(iters, cyc, sink);
+  rate_kernel<OP1, OP2><<<sms, THREADS>>>(iters, cyc, sink);
   cudaEventRecord(e1);
   const int rc = (cudaGetLastError() == cudaSuccess && cudaEventSynchronize(e1) == cudaSuccess) ? 0 : -2;
   if (rc == 0) cudaEventElapsedTime(ms, e0, e1);
@@ -127,7 +147,13 @@ extern "C" int mmaemu_peak_rate(int op, int iters, double *lanes_per_sm_clk, dou
     case PEAK_POPC: rc = run<PEAK_POPC>(iters, sms, cyc, sink, &ms); break;
     case PEAK_PRMT: rc = run<PEAK_PRMT>(iters, sms, cyc, sink, &ms); break;
     case PEAK_IMNMX: rc = run<PEAK_IMNMX>(iters, sms, cyc, sink, &ms); break;
-    default: rc = run<PEAK_FFMA>(iters, sms, cyc, sink, &ms); break;
+    case PEAK_FFMA: rc = run<PEAK_FFMA>(iters, sms, cyc, sink, &ms); break;
+    case PEAK_DFMA_LOP3: rc = run<PEAK_DFMA, PEAK_LOP3>(iters, sms, cyc, sink, &ms); break;
+    case PEAK_DFMA_IMAD: rc = run<PEAK_DFMA, PEAK_IMAD>(iters, sms, cyc, sink, &ms); break;
+    case PEAK_DFMA_FFMA: rc = run<PEAK_DFMA, PEAK_FFMA>(iters, sms, cyc, sink, &ms); break;
+    case PEAK_DFMA_ADDMIN2: rc = run<PEAK_DFMA, PEAK_ADDMIN2>(iters, sms, cyc, sink, &ms); break;
+    case PEAK_LOP3_IMAD: rc = run<PEAK_LOP3, PEAK_IMAD>(iters, sms, cyc, sink, &ms); break;
+    default: rc = run<PEAK_LOP3, PEAK_FFMA>(iters, sms, cyc, sink, &ms); break;
   }
   if (rc == 0) {
     unsigned long long host[1024];

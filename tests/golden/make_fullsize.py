@@ -172,38 +172,45 @@ def main() -> int:
     ap.add_argument("--tiles", action="store_true", help="store the tile workloads' digests")
     args = ap.parse_args()
 
-    data = {}
-    if os.path.exists(OUT):
-        with open(OUT) as fh:
-            data = json.load(fh)
-    data.setdefault("workloads", {})
-    data.setdefault("timings", {})
-    data.setdefault("tiles", {})
+    updates = {"workloads": {}, "timings": {}, "tiles": {}}
     if args.tiles:
-        data["tiles"].update(run_tiles(args.threads))
+        updates["tiles"].update(run_tiles(args.threads))
     elif args.time_python_tiles:
-        data["timings"]["python_oracle_tiles_4096"] = dict(time_python_tiles(), host=host_info())
+        updates["timings"]["python_oracle_tiles_4096"] = dict(time_python_tiles(), host=host_info())
     elif args.time_only:
         rec = run_one(args.time_only, args.threads)
-        want = data["workloads"].get(args.time_only)
+        want = load().get("workloads", {}).get(args.time_only)
         if want is not None and want["d_sha256"] != rec["d_sha256"]:
             raise SystemExit(f"{args.time_only}: result differs from the stored digest")
-        data["timings"][f"{args.time_only}-{args.threads}threads"] = {
+        updates["timings"][f"{args.time_only}-{args.threads}threads"] = {
             "seconds": rec["oracle_seconds"], "threads": args.threads, "macs_per_s": rec["oracle_macs_per_s"],
             "host": host_info()}
     else:
         for name in args.only or list(workloads()):
             rec = run_one(name, args.threads)
             rec["host"] = host_info()
-            data["workloads"][name] = rec
             print(name, rec["oracle_seconds"], "s", rec["specials"], flush=True)
-            with open(OUT, "w") as fh:
-                json.dump(data, fh, indent=1, sort_keys=True)
-                fh.write("\n")
+            save({"workloads": {name: rec}})
+    save(updates)
+    return 0
+
+
+def load() -> dict:
+    if os.path.exists(OUT):
+        with open(OUT) as fh:
+            return json.load(fh)
+    return {}
+
+
+def save(updates: dict) -> None:
+    """Merge into the file as it is now (other runs may have written to it
+    meanwhile)."""
+    data = load()
+    for sec, recs in updates.items():
+        data.setdefault(sec, {}).update(recs)
     with open(OUT, "w") as fh:
         json.dump(data, fh, indent=1, sort_keys=True)
         fh.write("\n")
-    return 0
 
 
 if __name__ == "__main__":

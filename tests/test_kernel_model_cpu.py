@@ -106,7 +106,8 @@ def test_kernel_design_on_tile_classes(cref, km, model, fmt):
 
 
 @pytest.mark.parametrize("mistake", ["MISTAKE_NO_COUNT", "MISTAKE_NO_SKEW", "MISTAKE_NO_MASK", "MISTAKE_NO_FLOOR",
-                                     "MISTAKE_SUBNORMAL_CODE", "MISTAKE_NEAREST_WRITEBACK"])
+                                     "MISTAKE_SUBNORMAL_CODE", "MISTAKE_NEAREST_WRITEBACK",
+                                     "MISTAKE_HOPPER_UNTRUNCATED"])
 def test_planted_mistakes_in_the_design_are_caught(cref, tmp_path, mistake):
     lib = model_lib(tmp_path, mistake)
     caught = False

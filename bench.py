@@ -354,16 +354,24 @@ def oracle_rows(rows: int, nthreads: int, inputs=None):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(target_s: float = 12.0, inputs=None):
+def sample_rows(seconds: float, nthreads: int, inputs) -> int:
+    """Output rows the oracle computes in about `seconds` on nthreads threads.
+    The oracle hands out whole rows to its threads, so the probe runs two
+    rows per thread (every thread busy) and the answer is a multiple of
+    nthreads."""
+    probe = 2 * nthreads
+    per_row = oracle_rows(probe, nthreads, inputs) / probe
+    rows = int(seconds / max(per_row, 1e-9)) // nthreads * nthreads
+    return int(max(nthreads, min(M, rows)))
+
+
+def cpu_baseline(target_s: float = 15.0, inputs=None):
     """Time the oracle as it stands on a bounded sample: the first R output
     rows of the same GEMM (R x 4096 x 4096 MACs), R sized for ~target_s."""
     from oracle import cref
 
     nthreads = cref.default_threads()
-    rows = max(1, nthreads // 4)
-    dt = oracle_rows(rows, nthreads, inputs)
-    est = dt / rows
-    rows = int(max(1, min(M, target_s / max(est, 1e-6))))
+    rows = sample_rows(target_s, nthreads, inputs)
     dt = oracle_rows(rows, nthreads, inputs)
     macs = rows * N * K
     return {"value": macs / dt, "unit": UNIT, "cores": nthreads, "kind": "oracle",
@@ -382,8 +390,7 @@ def run_reference(args):
     nthreads = cref.default_threads()
     steps, warmup = args.steps, args.warmup
     budget = 150.0  # seconds for the whole run
-    probe = oracle_rows(max(1, nthreads // 4), nthreads, inputs) / max(1, nthreads // 4)
-    rows = int(max(1, min(M, budget / (steps + warmup) / max(probe, 1e-6))))
+    rows = sample_rows(budget / (steps + warmup), nthreads, inputs)
     for _ in range(warmup):
         oracle_rows(rows, nthreads, inputs)
     times = [oracle_rows(rows, nthreads, inputs) for _ in range(steps)]

@@ -680,11 +680,12 @@ __device__ __forceinline__ uint32_t store_b8(PanelT &P, int n, int h, const Raw8
 
 // Fast decode of 8 k-consecutive elements (k = 8h .. 8h+7) of A row idx or
 // B column idx into a tile panel, for elements that hold no Inf or NaN
-// (has_special tells).  An element's bits shifted into the high word of a
-// double give its value times 2^(bias - 1023) exactly -- normals and
-// subnormals alike, since both formats mark subnormals the same way -- and
-// one multiply by 2^(1023 - bias) (times 1 + 2^-40 for B) restores it.  The
-// exponent codes and sign bits come from packed operations on element pairs.
+// (has_special tells).  Values come from exact hardware conversions (fp16
+// and, through its fp32 bit pattern, bf16 to fp64; e4m3 first to an exact
+// f16 pair), subnormals included.  The exponent codes and sign bits come
+// from packed operations on element pairs of the 16-bit form: for e4m3 that
+// form is fp16, whose exponent field is clamped below at 9 (e = -6, the e4m3
+// subnormal exponent) instead of 1.
 template <int FMT>
 __device__ __forceinline__ bool has_special(const Raw8<FMT> &raw) {
   using T = FmtT<FMT>;
@@ -700,63 +701,77 @@ __device__ __forceinline__ bool has_special(const Raw8<FMT> &raw) {
   return any != 0;
 }
 
+// two e4m3 (low byte first) to an fp16 pair, exactly
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t b16) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "r"(b16));
+  return r;
+}
+// an fp16 pair to two doubles, exactly
+__device__ __forceinline__ void f16x2_to_f64(uint32_t w, double &lo, double &hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f64.f16 %0, l;\n\tcvt.f64.f16 %1, h;\n\t}"
+      : "=d"(lo), "=d"(hi)
+      : "r"(w));
+}
+
 template <int FMT, bool ISB, class PanelT>
 __device__ __forceinline__ uint32_t fast_store8(PanelT &P, int idx, int h, const Raw8<FMT> &raw) {
-  using T = FmtT<FMT>;
-  constexpr double SCALE = pow2d(1023 - T::BIAS) * (ISB ? 1.0 + pow2d(-40) : 1.0);
-  uint32_t neg = 0, pos = 0;  // element 2j+b at bit 2j + 16b, before the offset h
-  if constexpr (T::NBITS == 16) {
-    constexpr int SH = T::P - 4;  // brings the element's field to the double's exponent bits
-    constexpr uint32_t VMASK = 0x80000000u | (((1u << (T::P + T::EBITS)) - 1u) << (20 - T::P));
-    constexpr uint32_t EM2 = ((1u << T::EBITS) - 1u) * 0x10001u;
-    constexpr uint32_t K2 = (uint32_t)((512 + T::BIAS) * 16) * 0x10001u;  // op_code(e) = K2 - 16 max(field, 1)
-    constexpr uint32_t QZ_ADD = (uint32_t)(QZ - (512 + T::BIAS - 1) * 16);
+  // the 16-bit form: bf16 as stored, fp16 as stored, e4m3 converted to fp16
+  constexpr bool BF = FMT == FMT_BF16;
+  constexpr int P16 = BF ? 7 : 10, BIAS16 = BF ? 127 : 15;
+  constexpr uint32_t EM2 = (BF ? 0xFFu : 0x1Fu) * 0x10001u;
+  constexpr uint32_t FMIN = FMT == FMT_E4M3 ? 9u : 1u;  // smallest exponent field (subnormal exponent)
+  // op_code(e) = K2 - 16 max(field, FMIN) for a nonzero element, QZ for a
+  // zero one (field 0, so max(field, FMIN) = FMIN): with z = 1 for nonzero,
+  // code = (K2 + QZ_ADD) - 16 max(field, FMIN) - z QZ_ADD, lane by lane
+  // (every lane stays in [0, 2^16), so nothing borrows across lanes)
+  constexpr uint32_t K2 = (uint32_t)(512 + BIAS16) * 16u;
+  constexpr uint32_t QZ_ADD = (uint32_t)QZ - K2 + 16u * FMIN;
+  constexpr uint32_t KQ = (K2 + QZ_ADD) * 0x10001u;
+  static_assert(K2 + QZ_ADD < 65536u && K2 > 16u * 255u, "codes stay inside their 16-bit lanes");
+  constexpr double GROW = 1.0 + pow2d(-40);
+  uint32_t w16[4];
+  if constexpr (FMT == FMT_E4M3) {
 #pragma unroll
-    for (int j = 0; j < 4; j++) {
-      const uint32_t w = raw.w[j];
-      const int k = 8 * h + 2 * j;
-      const uint32_t h0 = (uint32_t)((int32_t)__byte_perm(w, 0, 0x1044) >> SH) & VMASK;
-      const uint32_t h1 = (uint32_t)((int32_t)w >> SH) & VMASK;
-      const double v0 = __hiloint2double((int)h0, 0) * SCALE, v1 = __hiloint2double((int)h1, 0) * SCALE;
-      const uint32_t nz = ((w & 0x7FFF7FFFu) + 0x7FFF7FFFu) & 0x80008000u;  // element nonzero
-      uint32_t q2 = K2 - vmaxu2_16((w >> T::P) & EM2, 0x00010001u) * 16u;
-      q2 += ((nz ^ 0x80008000u) >> 15) * QZ_ADD;  // zeros: QZ
-      if constexpr (ISB) {
-        P.bV[k][PanelT::bslot(idx)] = v0;
-        P.bV[k + 1][PanelT::bslot(idx)] = v1;
-        P.bQ[k][idx] = (int16_t)(q2 & 0xFFFFu);
-        P.bQ[k + 1][idx] = (int16_t)(q2 >> 16);
-      } else {
-        P.aV[k][idx] = v0;
-        P.aV[k + 1][idx] = v1;
-        P.aQ2[k][idx] = __byte_perm(q2, 0, 0x1010);
-        P.aQ2[k + 1][idx] = __byte_perm(q2, 0, 0x3232);
-      }
-      neg |= (nz & w) >> (15 - 2 * j);
-      pos |= (nz & ~w) >> (15 - 2 * j);
-    }
+    for (int j = 0; j < 4; j++) w16[j] = e4m3x2_to_f16x2((raw.w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-      const uint32_t x = (raw.w[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-      const int k = 8 * h + i;
-      const uint32_t hv = (uint32_t)((int32_t)(x << 24) >> 7) & 0x80FE0000u;
-      const double v = __hiloint2double((int)hv, 0) * SCALE;
-      const uint32_t field = (x >> T::P) & 0xFu;
-      const bool nz = (x & 0x7Fu) != 0u;
-      const uint32_t q = nz ? (uint32_t)((512 + T::BIAS) * 16) - 16u * max(field, 1u) : (uint32_t)QZ;
-      if constexpr (ISB) {
-        P.bV[k][PanelT::bslot(idx)] = v;
-        P.bQ[k][idx] = (int16_t)q;
-      } else {
-        P.aV[k][idx] = v;
-        P.aQ2[k][idx] = q * 0x10001u;
-      }
-      const uint32_t at = (uint32_t)((i & 6) + 16 * (i & 1));
-      neg |= (uint32_t)(nz && (x >> 7)) << at;
-      pos |= (uint32_t)(nz && !(x >> 7)) << at;
-    }
+    for (int j = 0; j < 4; j++) w16[j] = raw.w[j];
   }
+  uint32_t sg = 0, nzw = 0;  // element 2j+b's sign / nonzero bit at bit 2j + 16b, before the offset h
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    const uint32_t w = w16[j];
+    const int k = 8 * h + 2 * j;
+    double v0, v1;
+    if constexpr (BF) {
+      v0 = (double)__uint_as_float(w << 16);
+      v1 = (double)__uint_as_float(w & 0xFFFF0000u);
+    } else {
+      f16x2_to_f64(w, v0, v1);
+    }
+    if constexpr (ISB) {
+      v0 *= GROW;  // exact
+      v1 *= GROW;
+    }
+    const uint32_t z = vminu2(w & 0x7FFF7FFFu, 0x00010001u);  // 1 per nonzero element
+    const uint32_t f = vmaxu2_16((w >> P16) & EM2, FMIN * 0x10001u);
+    const uint32_t q2 = KQ - 16u * f - QZ_ADD * z;
+    if constexpr (ISB) {
+      P.bV[k][PanelT::bslot(idx)] = v0;
+      P.bV[k + 1][PanelT::bslot(idx)] = v1;
+      P.bQ[k][idx] = (int16_t)(q2 & 0xFFFFu);
+      P.bQ[k + 1][idx] = (int16_t)(q2 >> 16);
+    } else {
+      P.aV[k][idx] = v0;
+      P.aV[k + 1][idx] = v1;
+      P.aQ2[k][idx] = __byte_perm(q2, 0, 0x1010);
+      P.aQ2[k + 1][idx] = __byte_perm(q2, 0, 0x3232);
+    }
+    sg |= (w >> (15 - 2 * j)) & (0x00010001u << (2 * j));
+    nzw |= z << (2 * j);
+  }
+  const uint32_t neg = sg & nzw, pos = ~sg & nzw;
   return ISB ? (pos << h) | (neg << (h + 8)) : (neg << h) | (pos << (h + 8));
 }
 

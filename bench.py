@@ -540,11 +540,15 @@ def run_gpu(args):
         count, first = mism.cpu().tolist()
         if count != 0:
             raise RuntimeError(f"verify mode found {count} mismatches (first at {first}) in its own result")
-        verified = {"verified": True, "against": "the call's own claimed D (verify mode), 0 mismatches"}
+        # and the claim itself (computed by the library) against the oracle's D
+        verified = verify_against_oracle(args.workload.rsplit("-verify", 1)[0], D.cpu().numpy(), None)
+        verified["against"] += "; the timed verify calls found 0 mismatches in that claim"
     elif mode in ("store", "wt", None) or spec["kind"] == "tiles":
         # the last timed call's result against the oracle's stored digests
+        # (only the plain GEMM call writes fingerprints here)
         base = args.workload[:-3] if mode == "wt" else args.workload  # B stored [N][K]: the same GEMM
-        verified = verify_against_oracle(base, D.cpu().numpy(), fp.cpu().numpy() if spec["kind"] == "gemm" else None)
+        verified = verify_against_oracle(base, D.cpu().numpy(),
+                                         fp.cpu().numpy() if spec["kind"] == "gemm" and mode == "store" else None)
     elif mode == "fponly":
         verified = {"verified": None, "against": "no stored oracle digest for this workload"}
         if GOLDEN_NAMES.get(args.workload.rsplit("-fponly", 1)[0]):

@@ -482,7 +482,15 @@ __device__ __forceinline__ void mma_chunk(const PanelT &P, int rl, int cl, doubl
     const int k0 = KN * st;
     group_codes<FMT, CHK, KN, CUNR>(P, rl, cl, k0, nm, sin);
     group_start<F>(P, rl, cl, X, nm, skew, gm);
-    group_products<KN, UNR>(P, rl, cl, k0, X);
+    if constexpr (NST == 1) {
+      // the last product outside the loop, so that the scheduler can run
+      // the write-back's integer work beside its FP64 multiply-adds
+      // (measured: Hopper BF16 GEMM 9.07 -> 8.93 ms; Ampere spills)
+      group_products<KN - 1, UNR>(P, rl, cl, k0, X);
+      group_products<1, 1>(P, rl, cl, k0 + KN - 1, X);
+    } else {
+      group_products<KN, UNR>(P, rl, cl, k0, X);
+    }
     if (st + 1 < NST) {
       hand_over<CHK, F>(X, nm);
       carry_codes<CHK>(X, nm);
@@ -895,12 +903,24 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 // one bulk copy of this GPU's global memory into this block's shared memory
-// (no multicast)
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
+// (no multicast), with an L2 cache policy (createpolicy) for the source lines
+__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
@@ -959,9 +979,12 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const Gemm
   auto issue_chunk = [&](int j) {
     GPanel &P = panels[j & 1];
     mbar_expect_tx(&bars[j & 1], (uint32_t)(ABLOB + BBLOB));
-    bulk_g2s(&P, p.dA + (blob_a0 + j) * ABLOB, (uint32_t)ABLOB, &bars[j & 1]);
-    bulk_g2s(reinterpret_cast<unsigned char *>(&P) + ABLOB, p.dB + (blob_b0 + j) * BBLOB, (uint32_t)BBLOB,
-             &bars[j & 1]);
+    // L2 policy: a block row's A blobs serve every column block of its
+    // group, a column's B blobs only the group's blocks in that column,
+    // which run at the same time (measured: DRAM traffic -11%, time equal)
+    bulk_g2s_hint(&P, p.dA + (blob_a0 + j) * ABLOB, (uint32_t)ABLOB, &bars[j & 1], policy_evict_last());
+    bulk_g2s_hint(reinterpret_cast<unsigned char *>(&P) + ABLOB, p.dB + (blob_b0 + j) * BBLOB, (uint32_t)BBLOB,
+                  &bars[j & 1], policy_evict_first());
   };
   auto parity = [](int j) { return (uint32_t)(j >> 1) & 1u; };
   if (tid == 0) {

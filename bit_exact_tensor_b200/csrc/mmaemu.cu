@@ -6,7 +6,7 @@
 //                    fp32 result feeding the next), fused per-tile xorsum;
 //                    operand panels decoded once per call (decode_a_kernel,
 //                    decode_b_kernel) and staged by bulk asynchronous copies.
-//   tiles_kernel  -- independent 16x16x16 tiles, one warp per tile.
+//   tiles_kernel  -- independent 16x16x16 tiles, two per warp (4 x 4 outputs a lane).
 //   xorsum_kernel -- XOR of a buffer of 32-bit words.
 // The arithmetic model and its exact-double formulation are described in
 // mmaemu_core.cuh.  Tensor cores are deliberately not used: B200's own MMA
@@ -1119,69 +1119,74 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const Gemm
 }
 
 // ---------------------------------------------------------------------------
-// independent tiles: one warp per 16x16x16 tile, each lane 2 x 4 outputs
+// independent tiles, two per warp: one per half-warp, each lane 4 x 4
+// outputs of its tile and the decode of one A row and one B column.  Against
+// one tile per warp with 2 x 4 outputs per lane (3 blocks per SM at 80
+// registers), this halves the shared loads per product and doubles each
+// lane's independent accumulators: 100k Ampere-FP16 tiles 0.143 -> 0.126 ms.
 // ---------------------------------------------------------------------------
-constexpr int TWARPS = 8, TR = 2, TCC = 4;
 using TPanel = Panel<16, 16>;
+constexpr int T4WARPS = 8;
 // resident blocks per SM and k-loop unroll of the tile kernel (measured)
-#ifndef MMAEMU_TMINB
-#define MMAEMU_TMINB 3
+#ifndef MMAEMU_T4MINB
+#define MMAEMU_T4MINB 2
 #endif
 #ifndef MMAEMU_TUNROLL
-#define MMAEMU_TUNROLL 8
+#define MMAEMU_TUNROLL 4
 #endif
-
 template <int MODEL, int FMT>
-__global__ void __launch_bounds__(TWARPS * 32, MMAEMU_TMINB) tiles_kernel(const void *__restrict__ A, const void *__restrict__ B,
-                                                            const float *__restrict__ C, float *__restrict__ Dout,
-                                                            size_t ntiles) {
+__global__ void __launch_bounds__(T4WARPS * 32, MMAEMU_T4MINB)
+    tiles_kernel(const void *__restrict__ A, const void *__restrict__ B, const float *__restrict__ C,
+                   float *__restrict__ Dout, size_t ntiles) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  TPanel &P = reinterpret_cast<TPanel *>(smem_raw)[warp];
-  const int rl = (lane >> 2) * TR, cl = (lane & 3) * TCC;
-  const int lm = lane & 15, lh = lane >> 4;
-  const size_t stride = (size_t)gridDim.x * TWARPS;
-  size_t t = (size_t)blockIdx.x * TWARPS + warp;
-  if (t >= ntiles) return;  // warp-uniform
+  const int half = lane >> 4, l16 = lane & 15;
+  TPanel &P = reinterpret_cast<TPanel *>(smem_raw)[2 * warp + half];
+  const int rl = (l16 >> 2) * 4, cl = (l16 & 3) * 4;
+  const size_t stride = (size_t)gridDim.x * T4WARPS * 2;
+  size_t w0 = ((size_t)blockIdx.x * T4WARPS + warp) * 2;  // this warp's first tile (warp-uniform)
+  if (w0 >= ntiles) return;
+  size_t t = w0 + half;
+  bool act = t < ntiles;  // the second half may have no tile at the end
 
-  // raw operands and C of the next tile are loaded while this one computes
-  auto load_a = [&](size_t u) { return load_row8<FMT>(A, u * 256 + lm * 16 + 8 * lh, true); };
-  auto load_b = [&](size_t u) { return load_col8<FMT>(B, u * 256 + (8 * lh) * 16 + lm, 16, true); };
-  auto load_c = [&](size_t u, uint32_t(&cv)[TR][TCC]) {
-    load_bits<TR, TCC>(C + (C != nullptr ? u * 256 + rl * 16 + cl : 0), 16, C != nullptr, cv);
+  auto load_a = [&](size_t u, int h, bool v) { return load_row8<FMT>(A, u * 256 + l16 * 16 + 8 * h, v); };
+  auto load_b = [&](size_t u, int h, bool v) { return load_col8<FMT>(B, u * 256 + (8 * h) * 16 + l16, 16, v); };
+  auto load_c = [&](size_t u, bool v, uint32_t(&cv)[4][4]) {
+    const bool have = C != nullptr && v;
+    load_bits<4, 4>(C + (have ? u * 256 + rl * 16 + cl : 0), 16, have, cv);
   };
-  Raw8<FMT> ra = load_a(t), rb = load_b(t);
-  uint32_t cnext[TR][TCC];
-  load_c(t, cnext);
-  double X[TR][TCC];
+  Raw8<FMT> ra0 = load_a(t, 0, act), ra1 = load_a(t, 1, act), rb0 = load_b(t, 0, act), rb1 = load_b(t, 1, act);
+  uint32_t cnext[4][4];
+  load_c(t, act, cnext);
+  double X[4][4];
   uint32_t dneg0;
   for (;;) {
     bool chk = init_states<FMT>(cnext, X, dneg0);
-    __syncwarp();  // the previous tile's reads of P are done
-    // operands: the fast packed decode unless the tile holds Inf or NaN
-    uint32_t sp = 0;
-    uint32_t abits, bbits;
-    if (!__any_sync(0xFFFFFFFFu, has_special<FMT>(ra) || has_special<FMT>(rb))) {
-      abits = fast_store8<FMT, false>(P, lm, lh, ra);
-      bbits = fast_store8<FMT, true>(P, lm, lh, rb);
+    __syncwarp();  // the previous tiles' reads of the panels are done
+    uint32_t sp = 0, aw, bw;
+    const bool sp_raw = has_special<FMT>(ra0) || has_special<FMT>(ra1) || has_special<FMT>(rb0) ||
+                        has_special<FMT>(rb1);
+    if (!__any_sync(0xFFFFFFFFu, sp_raw)) {
+      aw = fast_store8<FMT, false>(P, l16, 0, ra0) | fast_store8<FMT, false>(P, l16, 1, ra1);
+      bw = fast_store8<FMT, true>(P, l16, 0, rb0) | fast_store8<FMT, true>(P, l16, 1, rb1);
     } else {
-      abits = store_a8<FMT>(P, lm, lh, ra, sp);
-      bbits = store_b8<FMT>(P, lm, lh, rb, sp);
+      aw = store_a8<FMT>(P, l16, 0, ra0, sp) | store_a8<FMT>(P, l16, 1, ra1, sp);
+      bw = store_b8<FMT>(P, l16, 0, rb0, sp) | store_b8<FMT>(P, l16, 1, rb1, sp);
     }
-    // sign words: the two half-rows (half-columns) of a row (column) meet
-    const uint32_t aw = abits | __shfl_xor_sync(0xFFFFFFFFu, abits, 16);
-    const uint32_t bw = bbits | __shfl_xor_sync(0xFFFFFFFFu, bbits, 16);
-    if (lh == 0) {
-      P.aS[lm] = aw;
-      P.bS[lm] = bw;
-    }
+    P.aS[l16] = aw;
+    P.bS[l16] = bw;
+    // either tile's Inf/NaN sends both through the per-output special path,
+    // which finds no special output in a tile without them
     const bool panel_special = __any_sync(0xFFFFFFFFu, sp != 0);
     __syncwarp();
-    const size_t next = t + stride;
-    if (next < ntiles) {
-      ra = load_a(next);
-      rb = load_b(next);
-      load_c(next, cnext);
+    const size_t w_next = w0 + stride, next = t + stride;
+    const bool act_next = next < ntiles;
+    if (w_next < ntiles) {
+      ra0 = load_a(next, 0, act_next);
+      ra1 = load_a(next, 1, act_next);
+      rb0 = load_b(next, 0, act_next);
+      rb1 = load_b(next, 1, act_next);
+      load_c(next, act_next, cnext);
     }
     if constexpr (FMT == FMT_BF16) {
       bool unused = false;
@@ -1199,13 +1204,17 @@ __global__ void __launch_bounds__(TWARPS * 32, MMAEMU_TMINB) tiles_kernel(const 
         }
       }
     }
-    uint32_t D[TR][TCC];
+    uint32_t D[4][4];
     states_to_fp32<MODEL>(X, chk, dneg0, D);
+    if (act) {
 #pragma unroll
-    for (int i = 0; i < TR; i++)
-      *reinterpret_cast<uint4 *>(Dout + t * 256 + (rl + i) * 16 + cl) = make_uint4(D[i][0], D[i][1], D[i][2], D[i][3]);
+      for (int i = 0; i < 4; i++)
+        *reinterpret_cast<uint4 *>(Dout + t * 256 + (rl + i) * 16 + cl) = make_uint4(D[i][0], D[i][1], D[i][2], D[i][3]);
+    }
+    w0 = w_next;
     t = next;
-    if (t >= ntiles) break;
+    act = act_next;
+    if (w0 >= ntiles) break;
   }
 }
 
@@ -1676,18 +1685,20 @@ int run_gemm(int model, int fmt, mmaemu::GemmParams &p, long long batch) {
 
 template <int MODEL, int FMT>
 int launch_tiles(const void *A, const void *B, const float *C, float *D, size_t ntiles, int sms) {
-  const size_t smem = mmaemu::TWARPS * sizeof(mmaemu::TPanel);
+  const size_t smem = 2 * mmaemu::T4WARPS * sizeof(mmaemu::TPanel);
   auto kern = mmaemu::tiles_kernel<MODEL, FMT>;
+  constexpr int TPB = 2 * mmaemu::T4WARPS;  // tiles per block and pass
+  constexpr int THREADS = mmaemu::T4WARPS * 32;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return MMAEMU_ECUDA;
   int per_sm = 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, mmaemu::TWARPS * 32, smem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, smem) != cudaSuccess)
     return MMAEMU_ECUDA;
   if (per_sm < 1) per_sm = 1;
-  const size_t want = (ntiles + mmaemu::TWARPS - 1) / mmaemu::TWARPS;
+  const size_t want = (ntiles + TPB - 1) / TPB;
   const size_t cap = (size_t)sms * per_sm;
   const unsigned blocks = (unsigned)(want < cap ? want : cap);
-  kern<<<blocks, mmaemu::TWARPS * 32, smem, t_stream>>>(A, B, C, D, ntiles);
+  kern<<<blocks, THREADS, smem, t_stream>>>(A, B, C, D, ntiles);
   return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
 }
 

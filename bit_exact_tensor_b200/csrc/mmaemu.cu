@@ -509,26 +509,27 @@ __device__ __forceinline__ void mma_chunk(const PanelT &P, int rl, int cl, doubl
 // is the carried value itself, so every result stays normal (or zero), and
 // over any K < 2^31 the values stay below 2^101 (FP16 products are below
 // 2^32, E4M3 products below 2^18; truncation never rounds up).
-template <int FMT>
-__device__ __forceinline__ bool unchecked_ok(uint32_t c) {
-  const uint32_t field = (c >> 23) & 0xFFu;
-  return FMT != FMT_BF16 && ((c << 1) == 0u || field - 1u < 226u);
-}
+// (the range test, for a block: the largest |c| bit pattern below 2^100's,
+// the smallest nonzero one at least 2^-126's; zeros wrap to the top in
+// |c| - 1 and drop out of the minimum)
+constexpr uint32_t UNCHECKED_MAX_BITS = 0x71800000u, UNCHECKED_MIN_BITS = 0x00800000u;
 
 template <int FMT, int R, int CC>
 __device__ __forceinline__ bool init_states(const uint32_t (&cb)[R][CC], double (&X)[R][CC], uint32_t &dneg0) {
-  bool ok = FMT != FMT_BF16;
+  uint32_t amax = 0, amin1 = 0xFFFFFFFFu;
   dneg0 = 0;
 #pragma unroll
   for (int r = 0; r < R; r++)
 #pragma unroll
     for (int c = 0; c < CC; c++) {
-      const uint32_t v = cb[r][c];
-      ok = ok && unchecked_ok<FMT>(v);
+      const uint32_t v = cb[r][c], a = v & 0x7FFFFFFFu;
+      amax = max(amax, a);
+      amin1 = min(amin1, a - 1u);
       dneg0 |= (uint32_t)(v == 0x80000000u) << (r * CC + c);
       // exact; -0 becomes +0 (its sign lives in dneg0); Inf and NaN stay so
       X[r][c] = (double)(__uint_as_float(v) + 0.0f);
     }
+  const bool ok = FMT != FMT_BF16 && amax < UNCHECKED_MAX_BITS && amin1 >= UNCHECKED_MIN_BITS - 1u;
   if (!ok) {
 #pragma unroll
     for (int r = 0; r < R; r++)

@@ -514,8 +514,12 @@ __device__ __forceinline__ void mma_chunk(const PanelT &P, int rl, int cl, doubl
 // |c| - 1 and drop out of the minimum)
 constexpr uint32_t UNCHECKED_MAX_BITS = 0x71800000u, UNCHECKED_MIN_BITS = 0x00800000u;
 
+// track_neg0 = false: the caller knows that no output can end as -0 from
+// a -0 incoming value (every product of the chunk is nonzero), so the -0
+// mask starts empty.
 template <int FMT, int R, int CC>
-__device__ __forceinline__ bool init_states(const uint32_t (&cb)[R][CC], double (&X)[R][CC], uint32_t &dneg0) {
+__device__ __forceinline__ bool init_states(const uint32_t (&cb)[R][CC], double (&X)[R][CC], uint32_t &dneg0,
+                                            bool track_neg0 = true) {
   uint32_t amax = 0, amin1 = 0xFFFFFFFFu;
   dneg0 = 0;
 #pragma unroll
@@ -525,7 +529,7 @@ __device__ __forceinline__ bool init_states(const uint32_t (&cb)[R][CC], double 
       const uint32_t v = cb[r][c], a = v & 0x7FFFFFFFu;
       amax = max(amax, a);
       amin1 = min(amin1, a - 1u);
-      dneg0 |= (uint32_t)(v == 0x80000000u) << (r * CC + c);
+      if (track_neg0) dneg0 |= (uint32_t)(v == 0x80000000u) << (r * CC + c);
       // exact; -0 becomes +0 (its sign lives in dneg0); Inf and NaN stay so
       X[r][c] = (double)(__uint_as_float(v) + 0.0f);
     }
@@ -548,6 +552,13 @@ __device__ __forceinline__ void states_to_fp32(double (&X)[R][CC], bool chk, uin
     // unchecked states are +0 (a set dneg0 bit marks -0) or lie in the
     // normal fp32 range, where the conversion toward zero is the 24-bit
     // truncation (exact for a state that is truncated already)
+    if (dneg0 == 0u) {
+#pragma unroll
+      for (int r = 0; r < R; r++)
+#pragma unroll
+        for (int c = 0; c < CC; c++) D[r][c] = __float_as_uint(__double2float_rz(X[r][c]));
+      return;
+    }
 #pragma unroll
     for (int r = 0; r < R; r++)
 #pragma unroll
@@ -1162,7 +1173,6 @@ __global__ void __launch_bounds__(T4WARPS * 32, MMAEMU_T4MINB)
   double X[4][4];
   uint32_t dneg0;
   for (;;) {
-    bool chk = init_states<FMT>(cnext, X, dneg0);
     __syncwarp();  // the previous tiles' reads of the panels are done
     uint32_t sp = 0, aw, bw;
     const bool sp_raw = has_special<FMT>(ra0) || has_special<FMT>(ra1) || has_special<FMT>(rb0) ||
@@ -1179,6 +1189,12 @@ __global__ void __launch_bounds__(T4WARPS * 32, MMAEMU_T4MINB)
     // either tile's Inf/NaN sends both through the per-output special path,
     // which finds no special output in a tile without them
     const bool panel_special = __any_sync(0xFFFFFFFFu, sp != 0);
+    // -0 can only come out of an output whose 16 products are all zero; when
+    // every operand of both tiles is nonzero and finite (each sign word has
+    // a bit for every k) no output can, and the -0 mask is not kept
+    const bool all_nonzero = __all_sync(0xFFFFFFFFu, ((aw | (aw >> 8)) & 0x00FF00FFu) == 0x00FF00FFu &&
+                                                         ((bw | (bw >> 8)) & 0x00FF00FFu) == 0x00FF00FFu);
+    bool chk = init_states<FMT>(cnext, X, dneg0, !all_nonzero);
     __syncwarp();
     const size_t w_next = w0 + stride, next = t + stride;
     const bool act_next = next < ntiles;

@@ -156,3 +156,22 @@ def test_product_path_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert not pat.search(text), f
+
+
+class _FakeTensor:
+    def __init__(self, device):
+        import torch
+
+        self.device = torch.device(device)
+
+
+def test_binding_refuses_operands_on_different_devices():
+    """Every wrapper runs with its operands' device current; operands on two
+    devices (or off the GPU) are refused on the host, before any launch."""
+    import bit_exact_tensor_b200 as mm
+
+    assert str(mm._device_of(_FakeTensor("cuda:1"), None, _FakeTensor("cuda:1"))) == "cuda:1"
+    with pytest.raises(ValueError):
+        mm._device_of(_FakeTensor("cuda:0"), _FakeTensor("cuda:1"))
+    with pytest.raises(TypeError):
+        mm._device_of(_FakeTensor("cpu"))

@@ -699,28 +699,13 @@ __device__ __forceinline__ uint32_t store_b8(PanelT &P, int n, int h, const Raw8
 }
 
 // Fast decode of 8 k-consecutive elements (k = 8h .. 8h+7) of A row idx or
-// B column idx into a tile panel, for elements that hold no Inf or NaN
-// (has_special tells).  Values come from exact hardware conversions (fp16
+// B column idx into a tile panel, right for elements that hold no Inf or NaN
+// (the caller tests fmax afterwards and decodes such tiles again).  Values come from exact hardware conversions (fp16
 // and, through its fp32 bit pattern, bf16 to fp64; e4m3 first to an exact
 // f16 pair), subnormals included.  The exponent codes and sign bits come
 // from packed operations on element pairs of the 16-bit form: for e4m3 that
 // form is fp16, whose exponent field is clamped below at 9 (e = -6, the e4m3
 // subnormal exponent) instead of 1.
-template <int FMT>
-__device__ __forceinline__ bool has_special(const Raw8<FMT> &raw) {
-  using T = FmtT<FMT>;
-  uint32_t any = 0;
-  if constexpr (T::NBITS == 16) {
-    constexpr uint32_t FM = (((1u << T::EBITS) - 1u) << T::P) * 0x10001u, ONE = (1u << T::P) * 0x10001u;
-#pragma unroll
-    for (int j = 0; j < 4; j++) any |= ((raw.w[j] & FM) + ONE) & 0x80008000u;  // field all ones
-  } else {
-#pragma unroll
-    for (int j = 0; j < 2; j++) any |= ((raw.w[j] & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;  // S.1111.111
-  }
-  return any != 0;
-}
-
 // two e4m3 (low byte first) to an fp16 pair, exactly
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t b16) {
   uint32_t r;
@@ -734,8 +719,10 @@ __device__ __forceinline__ void f16x2_to_f64(uint32_t w, double &lo, double &hi)
       : "r"(w));
 }
 
+// fmax: the running packed maximum of the 16-bit form's exponent fields,
+// for the caller's Inf/NaN test after the fact (a field of all ones).
 template <int FMT, bool ISB, class PanelT>
-__device__ __forceinline__ uint32_t fast_store8(PanelT &P, int idx, int h, const Raw8<FMT> &raw) {
+__device__ __forceinline__ uint32_t fast_store8(PanelT &P, int idx, int h, const Raw8<FMT> &raw, uint32_t &fmax) {
   // the 16-bit form: bf16 as stored, fp16 as stored, e4m3 converted to fp16
   constexpr bool BF = FMT == FMT_BF16;
   constexpr int P16 = BF ? 7 : 10, BIAS16 = BF ? 127 : 15;
@@ -776,6 +763,7 @@ __device__ __forceinline__ uint32_t fast_store8(PanelT &P, int idx, int h, const
     }
     const uint32_t z = vminu2(w & 0x7FFF7FFFu, 0x00010001u);  // 1 per nonzero element
     const uint32_t f = vmaxu2_16((w >> P16) & EM2, FMIN * 0x10001u);
+    fmax = vmaxu2_16(fmax, f);
     const uint32_t q2 = KQ - 16u * f - QZ_ADD * z;
     if constexpr (ISB) {
       P.bV[k][PanelT::bslot(idx)] = v0;
@@ -1175,14 +1163,20 @@ __global__ void __launch_bounds__(T4WARPS * 32, MMAEMU_T4MINB)
   for (;;) {
     __syncwarp();  // the previous tiles' reads of the panels are done
     uint32_t sp = 0, aw, bw;
-    const bool sp_raw = has_special<FMT>(ra0) || has_special<FMT>(ra1) || has_special<FMT>(rb0) ||
-                        has_special<FMT>(rb1);
-    if (!__any_sync(0xFFFFFFFFu, sp_raw)) {
-      aw = fast_store8<FMT, false>(P, l16, 0, ra0) | fast_store8<FMT, false>(P, l16, 1, ra1);
-      bw = fast_store8<FMT, true>(P, l16, 0, rb0) | fast_store8<FMT, true>(P, l16, 1, rb1);
-    } else {
-      aw = store_a8<FMT>(P, l16, 0, ra0, sp) | store_a8<FMT>(P, l16, 1, ra1, sp);
-      bw = store_b8<FMT>(P, l16, 0, rb0, sp) | store_b8<FMT>(P, l16, 1, rb1, sp);
+    // fast decode first; a tile pair whose operands hold Inf or NaN (an
+    // exponent field of all ones in the 16-bit form) is decoded again
+    // element by element, over the fast decode's panel entries
+    {
+      constexpr uint32_t EMAX = (FMT == FMT_BF16 ? 0xFFu : 0x1Fu) * 0x10001u;
+      uint32_t fmax = 0;
+      aw = fast_store8<FMT, false>(P, l16, 0, ra0, fmax) | fast_store8<FMT, false>(P, l16, 1, ra1, fmax);
+      bw = fast_store8<FMT, true>(P, l16, 0, rb0, fmax) | fast_store8<FMT, true>(P, l16, 1, rb1, fmax);
+      const bool special_here = (fmax & 0xFFFFu) == (EMAX & 0xFFFFu) || (fmax >> 16) == (EMAX >> 16);
+      if (__any_sync(0xFFFFFFFFu, special_here)) {
+        __syncwarp();
+        aw = store_a8<FMT>(P, l16, 0, ra0, sp) | store_a8<FMT>(P, l16, 1, ra1, sp);
+        bw = store_b8<FMT>(P, l16, 0, rb0, sp) | store_b8<FMT>(P, l16, 1, rb1, sp);
+      }
     }
     P.aS[l16] = aw;
     P.bS[l16] = bw;

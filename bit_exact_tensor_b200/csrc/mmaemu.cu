@@ -98,11 +98,12 @@ __device__ __forceinline__ bool neg_b(const PanelT &P, int k, int n) {
   return __double2hiint(P.bV[k][PanelT::bslot(n)]) < 0;
 }
 
-// Unroll of the GEMM's product loops, measured: 2 for Ampere FP16, 4 for
-// the rest (Ampere's exponent pass is unrolled fully, see mma_chunk).
+// Unroll of the GEMM's product loops, measured per model and format:
+// Ampere FP16 2, BF16 4; the one-stage models 8 for FP16 and E4M3, 4 for
+// BF16 (Ampere's exponent pass is unrolled fully, see mma_chunk).
 #ifndef MMAEMU_KUNROLL
 template <int MODEL, int FMT>
-constexpr int kUnroll = MODEL == MODEL_AMPERE && FMT == FMT_FP16 ? 2 : 4;
+constexpr int kUnroll = MODEL == MODEL_AMPERE ? (FMT == FMT_FP16 ? 2 : 4) : (FMT == FMT_BF16 ? 4 : 8);
 #else
 template <int MODEL, int FMT>
 constexpr int kUnroll = MMAEMU_KUNROLL;
@@ -500,10 +501,11 @@ __device__ __forceinline__ void mma_chunk(const PanelT &P, int rl, int cl, doubl
     const int k0 = KN * st;
     group_codes<FMT, CHK, KN, CUNR>(P, rl, cl, k0, nm, sin);
     group_start<F>(P, rl, cl, X, nm, skew, gm);
-    if constexpr (NST == 1) {
+    if constexpr (NST == 1 || FMT == FMT_FP16) {
       // the last product outside the loop, so that the scheduler can run
-      // the write-back's integer work beside its FP64 multiply-adds
-      // (measured: Hopper BF16 GEMM 9.07 -> 8.93 ms; Ampere spills)
+      // the write-back's (or hand-over's) integer work beside its FP64
+      // multiply-adds (measured: faster for the one-stage models and Ampere
+      // FP16, slower for Ampere BF16)
       group_products<KN - 1, UNR>(P, rl, cl, k0, X);
       group_products<1, 1>(P, rl, cl, k0 + KN - 1, X);
     } else {

@@ -509,17 +509,28 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
 
     def timed():
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        barrier()
-        torch.cuda.synchronize(dev)
+        """K steps between a barrier and a synchronisation, timed by events
+        around the whole run (the value), then K more with an event pair
+        around each call (each launch's duration, for the roofline).  The
+        first pass records nothing between steps: for the short tile batches
+        the per-step event records cost enough host time to leave the GPU
+        idle between calls."""
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
         t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
         for s, e in ev:
             s.record(stream)
             step()
             e.record(stream)
-        t1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
         per = [s.elapsed_time(e) for s, e in ev]

@@ -27,7 +27,10 @@
 //    truncation;
 //  * the exact group value is acc minus the base 1.5 * 2^52 u, one
 //    subtraction; truncating it to 24 significant bits is a mask of the low
-//    29 mantissa bits: the Ampere hand-over and the fp32 write-back.
+//    29 mantissa bits: the Ampere hand-over and the fp32 write-back (the
+//    unchecked Ampere form carries the exact value instead and truncates
+//    once at the end, which gives the same result: the next group's grid is
+//    never finer than the carried value's 24-bit unit).
 #pragma once
 #include <stdint.h>
 

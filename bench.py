@@ -547,10 +547,15 @@ def run_gpu(args):
     total_ms = max_over_ranks(total_ms)
     kern_ms = max_over_ranks(sum(per_ms) / len(per_ms))
 
-    if mode == "verify":  # the claim must verify clean
+    if mode == "verify":  # on every rank, the claim must verify clean
         count, first = mism.cpu().tolist()
         if count != 0:
             raise RuntimeError(f"verify mode found {count} mismatches (first at {first}) in its own result")
+    if rank != 0:
+        # every rank draws its own inputs (seed + 1000 rank); the stored
+        # oracle digests describe rank 0's, so rank 0 alone compares with them
+        verified = {"verified": None, "against": "checked on rank 0 (the stored digests are of its inputs)"}
+    elif mode == "verify":
         # and the claim itself (computed by the library) against the oracle's D
         verified = verify_against_oracle(args.workload.rsplit("-verify", 1)[0], D.cpu().numpy(), None)
         verified["against"] += "; the timed verify calls found 0 mismatches in that claim"

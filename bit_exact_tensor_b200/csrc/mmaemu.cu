@@ -1563,23 +1563,57 @@ int host_streams(cudaStream_t &in, cudaStream_t &out, cudaStream_t &compute2) {
   return MMAEMU_OK;
 }
 
+// Row boundaries of mmaemu_gemm_host's slabs, at multiples of GBM rows:
+// r0[0] = 0 < r0[1] < ... < r0[n] = M; returns n.  The first slab holds one
+// full wave of GEMM blocks (sms x MMAEMU_GMINB), the fewest rows that keep
+// every SM busy while the next slab is copied: nothing computes until B and
+// that slab have arrived.  The last slab is short, since its D is the one
+// copy left once computing ends.  The rows between go in up to
+// kHostMidSlabs equal slabs.
+constexpr int kHostMaxSlabs = 8, kHostMidSlabs = 4, kHostTailDiv = 16;
+int host_slabs(int M, int N, int sms, int *r0) {
+  const int nb = (M + mmaemu::GBM - 1) / mmaemu::GBM;  // row blocks
+  const int cb = (N + mmaemu::GBN - 1) / mmaemu::GBN;  // column blocks
+  const long long wave = (long long)sms * MMAEMU_GMINB;
+  int head = (int)((wave + cb - 1) / cb);
+  if (head < 1) head = 1;
+  if (head > nb) head = nb;
+  int n = 0, b = 0;
+  r0[0] = 0;
+  auto cut = [&](int blocks) {
+    b += blocks;
+    r0[++n] = b * mmaemu::GBM < M ? b * mmaemu::GBM : M;
+  };
+  cut(head);
+  const int rest = nb - head;
+  int tail = nb / kHostTailDiv > 1 ? nb / kHostTailDiv : 1;
+  if (tail > rest) tail = rest;
+  const int mid = rest - tail, nm = mid < kHostMidSlabs ? mid : kHostMidSlabs;
+  for (int i = 0; i < nm; i++) cut(mid / nm + (i < mid % nm));
+  if (tail > 0) cut(tail);
+  return n;
+}
+
 // mmaemu_gemm from host memory: B is copied and decoded once; A and C go in
-// row slabs (a multiple of 64 rows) on a copy stream while earlier slabs
-// compute, alternately on the caller's stream and a second compute stream
-// (so that one slab's last partial wave of blocks overlaps the next slab),
-// and each slab's D (and fingerprints) returns on another copy stream as
-// soon as that slab is done.
+// row slabs (host_slabs) on a copy stream while earlier slabs compute,
+// alternately on the caller's stream and a second compute stream (so that
+// one slab's last partial wave of blocks overlaps the next slab), and each
+// slab's D (and fingerprints) returns on another copy stream as soon as
+// that slab is done.
 template <int MODEL, int FMT>
 int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, const float *C_h, float *D_h,
-                     uint32_t *fp_h) {
+                     uint32_t *fp_h, int sms) {
   constexpr size_t ES = FMT == mmaemu::FMT_E4M3 ? 1 : 2;
   cudaStream_t s_in, s_out, c2;
   int rc = host_streams(s_in, s_out, c2);
   if (rc != MMAEMU_OK) return rc;
   const cudaStream_t cs[2] = {t_stream, c2};
-  const int rows_per = ((M + 7) / 8 + mmaemu::GBM - 1) / mmaemu::GBM * mmaemu::GBM;
-  const int nslab = (M + rows_per - 1) / rows_per;
-  const GemmSizes zs = gemm_sizes(rows_per, N, K, 1), zb = gemm_sizes(M, N, K, 1);
+  int r0s[kHostMaxSlabs + 1];
+  const int nslab = host_slabs(M, N, sms, r0s);
+  int max_rows = 0;
+  for (int sl = 0; sl < nslab; sl++)
+    if (r0s[sl + 1] - r0s[sl] > max_rows) max_rows = r0s[sl + 1] - r0s[sl];
+  const GemmSizes zs = gemm_sizes(max_rows, N, K, 1), zb = gemm_sizes(M, N, K, 1);
   const size_t a_bytes = (size_t)M * K * ES, b_bytes = (size_t)K * N * ES, cd_bytes = (size_t)M * N * 4;
   const size_t fp_bytes = fp_h ? (size_t)(M / 16) * (N / 16) * 4 : 0;
   // device buffers, each 256-byte aligned inside one pool allocation; two
@@ -1597,7 +1631,7 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
   uint32_t *dfp = fp_h ? reinterpret_cast<uint32_t *>(buf + o_fp) : nullptr;
 
   const int nev = 2 + 2 * nslab + 3;
-  cudaEvent_t ev[2 + 2 * 8 + 3];
+  cudaEvent_t ev[2 + 2 * kHostMaxSlabs + 3];
   int made = 0;
   for (; made < nev; made++)
     if (cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming) != cudaSuccess) {
@@ -1616,7 +1650,7 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
       ok(cudaMemcpyAsync(dB, B_h, b_bytes, cudaMemcpyHostToDevice, s_in)))
     ok(cudaEventRecord(e_b, s_in));
   for (int sl = 0; sl < nslab && rc == MMAEMU_OK; sl++) {
-    const size_t r0 = (size_t)sl * rows_per, rows = (size_t)(sl + 1 < nslab ? rows_per : M - (int)r0);
+    const size_t r0 = r0s[sl], rows = r0s[sl + 1] - r0s[sl];
     if (!ok(cudaMemcpyAsync(dA + r0 * K * ES, static_cast<const unsigned char *>(A_h) + r0 * K * ES, rows * K * ES,
                             cudaMemcpyHostToDevice, s_in)))
       break;
@@ -1631,8 +1665,8 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
   if (rc == MMAEMU_OK && ok(cudaStreamWaitEvent(t_stream, e_b, 0))) rc = launch_decode_b<MODEL, FMT>(p, 1, t_stream);
   if (rc == MMAEMU_OK && ok(cudaEventRecord(e_bdec, t_stream))) ok(cudaStreamWaitEvent(c2, e_bdec, 0));
   for (int sl = 0; sl < nslab && rc == MMAEMU_OK; sl++) {
-    const size_t r0 = (size_t)sl * rows_per;
-    const int rows = sl + 1 < nslab ? rows_per : M - (int)r0;
+    const size_t r0 = r0s[sl];
+    const int rows = r0s[sl + 1] - r0s[sl];
     const cudaStream_t st = cs[sl & 1];
     mmaemu::GemmParams q = p;
     q.M = rows;
@@ -1819,9 +1853,10 @@ int mmaemu_gemm_host(int model, int fmt, int M, int N, int K, const void *A, con
   mmaemu::GemmParams p = row_major_params(M, N, K, A, B, C, D, fingerprint_out);
   int rc = validate_gemm(p, 1);
   if (rc != MMAEMU_OK) return rc;
-  rc = check_device();
+  int sms = 0;
+  rc = check_device(&sms);
   if (rc != MMAEMU_OK) return rc;
-#define CALL_HOST(M_, F_) launch_gemm_host<M_, F_>(M, N, K, A, B, C, D, fingerprint_out)
+#define CALL_HOST(M_, F_) launch_gemm_host<M_, F_>(M, N, K, A, B, C, D, fingerprint_out, sms)
   MMAEMU_DISPATCH(model, fmt, CALL_HOST);
 #undef CALL_HOST
 }

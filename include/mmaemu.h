@@ -168,10 +168,12 @@ int mmaemu_gemm_strided_batched(int model, int fmt, int trans_a, int trans_b, in
  * and the results D and fingerprint_out (either may be NULL, not both) are
  * host pointers; layouts and rules as mmaemu_gemm.  The call copies B and
  * decodes it once, then streams A and C to the device in row slabs on a
- * library-owned copy stream while earlier slabs compute on the selected
- * stream, and copies each slab's D and fingerprints back on a second copy
- * stream as soon as that slab is done -- the transfers overlap the
- * arithmetic.  Page-locked host memory lets the copies run asynchronously;
+ * library-owned copy stream while earlier slabs compute, alternately on the
+ * selected stream and a library-owned second compute stream, and copies
+ * each slab's D and fingerprints back on another copy stream as soon as
+ * that slab is done -- the transfers overlap the arithmetic.  The first
+ * slab is one wave of GEMM blocks (so a GEMM with fewer blocks than the
+ * GPU holds at once runs as one slab), the last is short, at most six.  Page-locked host memory lets the copies run asynchronously;
  * other host memory works too, with the copies no longer overlapped.
  * Device memory comes from the library's workspace pool (see the GEMM
  * implementation note).  Returns after D and the fingerprints are in host

@@ -121,12 +121,15 @@ def test_workspace_is_released_by_default_and_cached_on_request(cref):
     assert mmaemu.workspace_reserved() == 0
 
 
-@pytest.mark.parametrize("shape", [(80, 144, 48), (1040, 400, 96), (64, 16, 16)], ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("shape", [(80, 144, 48), (1040, 400, 96), (64, 16, 16), (1040, 4096, 32)],
+                         ids=lambda s: "x".join(map(str, s)))
 @pytest.mark.parametrize("pinned", [True, False])
 def test_gemm_from_host_memory(cref, shape, pinned):
     """mmaemu_gemm_host: host buffers in and out, A/C/D streamed in row
-    slabs (1040 rows: five slabs of 192 and one of 80) overlapped with the
-    arithmetic -- the same bits as the device call and the oracle."""
+    slabs overlapped with the arithmetic -- the same bits as the device call
+    and the oracle.  The first slab holds one wave of GEMM blocks, so the
+    narrow shapes run as one slab; 1040 x 4096 on 148 SMs runs as six
+    (640 rows, then 128, 128, 64, 64, and a ragged last slab of 16)."""
     import torch
 
     import bit_exact_tensor_b200 as mmaemu

@@ -19,7 +19,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "mmaemu.cu")
 SOURCES = [SRC, os.path.join(PKG, "csrc", "probe.cpp")]
-DEPS = SOURCES + [os.path.join(PKG, "csrc", "mmaemu_core.cuh"), os.path.join(ROOT, "include", "mmaemu.h"),
+DEPS = SOURCES + [os.path.join(PKG, "csrc", "mmaemu_core.cuh"), os.path.join(PKG, "csrc", "host_slabs.h"),
+                  os.path.join(ROOT, "include", "mmaemu.h"),
                   os.path.join(ROOT, "include", "mmaemu_probe.h"), os.path.abspath(__file__)]
 LIB = os.path.join(PKG, "libmmaemu.so")
 LIB_CHECK = os.path.join(PKG, "libmmaemu_check.so")

@@ -19,6 +19,7 @@
 
 #include "mmaemu.h"
 #include "mmaemu_core.cuh"
+#include "host_slabs.h"
 
 namespace mmaemu {
 
@@ -1563,39 +1564,8 @@ int host_streams(cudaStream_t &in, cudaStream_t &out, cudaStream_t &compute2) {
   return MMAEMU_OK;
 }
 
-// Row boundaries of mmaemu_gemm_host's slabs, at multiples of GBM rows:
-// r0[0] = 0 < r0[1] < ... < r0[n] = M; returns n.  The first slab holds one
-// full wave of GEMM blocks (sms x MMAEMU_GMINB), the fewest rows that keep
-// every SM busy while the next slab is copied: nothing computes until B and
-// that slab have arrived.  The last slab is short, since its D is the one
-// copy left once computing ends.  The rows between go in up to
-// kHostMidSlabs equal slabs.
-constexpr int kHostMaxSlabs = 8, kHostMidSlabs = 4, kHostTailDiv = 16;
-int host_slabs(int M, int N, int sms, int *r0) {
-  const int nb = (M + mmaemu::GBM - 1) / mmaemu::GBM;  // row blocks
-  const int cb = (N + mmaemu::GBN - 1) / mmaemu::GBN;  // column blocks
-  const long long wave = (long long)sms * MMAEMU_GMINB;
-  int head = (int)((wave + cb - 1) / cb);
-  if (head < 1) head = 1;
-  if (head > nb) head = nb;
-  int n = 0, b = 0;
-  r0[0] = 0;
-  auto cut = [&](int blocks) {
-    b += blocks;
-    r0[++n] = b * mmaemu::GBM < M ? b * mmaemu::GBM : M;
-  };
-  cut(head);
-  const int rest = nb - head;
-  int tail = nb / kHostTailDiv > 1 ? nb / kHostTailDiv : 1;
-  if (tail > rest) tail = rest;
-  const int mid = rest - tail, nm = mid < kHostMidSlabs ? mid : kHostMidSlabs;
-  for (int i = 0; i < nm; i++) cut(mid / nm + (i < mid % nm));
-  if (tail > 0) cut(tail);
-  return n;
-}
-
 // mmaemu_gemm from host memory: B is copied and decoded once; A and C go in
-// row slabs (host_slabs) on a copy stream while earlier slabs compute,
+// row slabs (host_slabs.h) on a copy stream while earlier slabs compute,
 // alternately on the caller's stream and a second compute stream (so that
 // one slab's last partial wave of blocks overlaps the next slab), and each
 // slab's D (and fingerprints) returns on another copy stream as soon as
@@ -1608,8 +1578,8 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
   int rc = host_streams(s_in, s_out, c2);
   if (rc != MMAEMU_OK) return rc;
   const cudaStream_t cs[2] = {t_stream, c2};
-  int r0s[kHostMaxSlabs + 1];
-  const int nslab = host_slabs(M, N, sms, r0s);
+  int r0s[mmaemu_host::kHostMaxSlabs + 1];
+  const int nslab = mmaemu_host::host_slabs(M, N, mmaemu::GBM, mmaemu::GBN, (long long)sms * MMAEMU_GMINB, r0s);
   int max_rows = 0;
   for (int sl = 0; sl < nslab; sl++)
     if (r0s[sl + 1] - r0s[sl] > max_rows) max_rows = r0s[sl + 1] - r0s[sl];
@@ -1631,7 +1601,7 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
   uint32_t *dfp = fp_h ? reinterpret_cast<uint32_t *>(buf + o_fp) : nullptr;
 
   const int nev = 2 + 2 * nslab + 3;
-  cudaEvent_t ev[2 + 2 * kHostMaxSlabs + 3];
+  cudaEvent_t ev[2 + 2 * mmaemu_host::kHostMaxSlabs + 3];
   int made = 0;
   for (; made < nev; made++)
     if (cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming) != cudaSuccess) {

@@ -230,6 +230,25 @@ def verify_against_oracle(name, D_host, fp_host):
     return out
 
 
+def verify_fp_against_oracle(name, fp_host):
+    """The fingerprint-only mode's result against the oracle's stored
+    fingerprint digest; raises on a difference."""
+    import hashlib
+
+    import numpy as np
+
+    if not GOLDEN_NAMES.get(name) or not os.path.exists(GOLDEN):
+        return {"verified": None, "against": "no stored oracle digest for this workload"}
+    sec, key = GOLDEN_NAMES[name]
+    with open(GOLDEN) as fh:
+        want = json.load(fh)[sec][key]["fp_sha256"]
+    got = hashlib.sha256(np.ascontiguousarray(fp_host.view(np.uint32), dtype="<u4").tobytes())
+    out = {"verified": got.hexdigest() == want, "against": f"oracle fingerprint digest [{sec}][{key}]"}
+    if not out["verified"]:
+        raise RuntimeError("fingerprints differ from the oracle's")
+    return out
+
+
 def run_pipe_rates():
     """Print the measured issue rates of the instruction classes the kernels
     use, with the SM clock sampled during the probes."""
@@ -566,17 +585,7 @@ def run_gpu(args):
         verified = verify_against_oracle(base, D.cpu().numpy(),
                                          fp.cpu().numpy() if spec["kind"] == "gemm" and mode == "store" else None)
     elif mode == "fponly":
-        verified = {"verified": None, "against": "no stored oracle digest for this workload"}
-        if GOLDEN_NAMES.get(args.workload.rsplit("-fponly", 1)[0]):
-            import hashlib
-
-            sec, key = GOLDEN_NAMES[args.workload.rsplit("-fponly", 1)[0]]
-            with open(GOLDEN) as fh:
-                want = json.load(fh)[sec][key]["fp_sha256"]
-            got = hashlib.sha256(np.ascontiguousarray(fp.cpu().numpy().view(np.uint32), dtype="<u4").tobytes())
-            verified = {"verified": got.hexdigest() == want, "against": f"oracle fingerprint digest [{sec}][{key}]"}
-            if not verified["verified"]:
-                raise RuntimeError("fingerprints differ from the oracle's")
+        verified = verify_fp_against_oracle(args.workload.rsplit("-fponly", 1)[0], fp.cpu().numpy())
     else:
         verified = {"verified": None, "against": "no stored oracle digest for this workload"}
     # issue rates of the FP64 pipe and of the fastest INT32 instruction,
@@ -624,13 +633,34 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    last = None
     e0.record(stream)
     for _ in range(args.e2e_steps):
-        e2e_step()
+        # the previous result is released first, so that its page-locked
+        # buffers go back to the host allocator's cache for this call
+        last = None
+        last = e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps)
     barrier()
+    # the last end-to-end call's result, in host memory, against the same
+    # oracle digests (rank 0, after the timed region)
+    e2e_verified = None
+    if rank == 0 and last is not None:
+        Dh, fph = last
+        if mode == "verify":
+            count = int(Dh.view(-1)[0])
+            e2e_verified = count == 0
+            if count != 0:
+                raise RuntimeError(f"the end-to-end verify call found {count} mismatches in the oracle-equal claim")
+        elif mode == "fponly":
+            e2e_verified = verify_fp_against_oracle(args.workload.rsplit("-fponly", 1)[0], fph.numpy())["verified"]
+        else:
+            base = args.workload[:-3] if mode == "wt" else args.workload
+            e2e_verified = verify_against_oracle(
+                base, Dh.numpy(), fph.numpy() if spec["kind"] == "gemm" and mode == "store" and fph is not None
+                else None)["verified"]
 
     if rank == 0:
         macs = spec["macs"]
@@ -682,7 +712,7 @@ def run_gpu(args):
             "roofline": roof,
             "clocks": clocks,
             "e2e": {"value": macs * world / (e2e_ms / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "verified": e2e_verified},
             "gpu_launches": launches_per_step * args.steps,
         }
         if world == 1 and not args.no_cpu_baseline and args.workload == DEFAULT_WORKLOAD:

@@ -225,6 +225,30 @@ def test_full_size_equals_the_oracle_everywhere(name):
     assert int(np.bitwise_xor.reduce(D.ravel())) == rec["xorsum"]
 
 
+@pytest.mark.parametrize("name", ["cfg3-ampere-fp16-4096", "cfg5-hopper-e4m3-8192x4096x14336"])
+def test_full_size_from_host_memory_equals_the_oracle(name):
+    """mmaemu_gemm_host, the call the end-to-end benchmark times, at full
+    size from page-locked host buffers: every element of D and every tile
+    fingerprint equals the oracle's (its row slabs and two compute streams
+    change nothing)."""
+    import torch
+
+    import bit_exact_tensor_b200 as mmaemu
+
+    model, fmt, make = FULL[name]
+    rec = golden_record(name)
+    A, B, C = make()
+
+    def host(x):
+        v = x.view(np.uint8) if x.dtype == np.uint8 else x.view(np.int16) if x.dtype == np.uint16 else x.view(np.int32)
+        return torch.from_numpy(v).pin_memory()
+
+    D, fp = mmaemu.gemm_host(model, fmt, host(A), host(B), host(C))
+    got = fullsize_digests(D.view(torch.int32).numpy().view(np.uint32), fp.numpy().view(np.uint32))
+    assert got["d_sha256"] == rec["d_sha256"], "D from host memory differs from the oracle's"
+    assert got["fp_sha256"] == rec["fp_sha256"], "tile fingerprints from host memory differ from the oracle's"
+
+
 def test_full_size_deterministic():
     A, B, C = wl.config3()
     _, fp1 = run_gemm("ampere", "fp16", A, B, C)

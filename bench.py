@@ -598,6 +598,10 @@ def run_gpu(args):
     C_h = torch.from_numpy(C_np.view(np.int32)).pin_memory()
     if mode == "verify":
         Dclaim_h = D.cpu().pin_memory()
+    if mode == "store":  # the results land in page-locked buffers owned by the caller
+        D_out_h = torch.empty(C_h.shape, dtype=torch.float32, pin_memory=True)
+        fp_out_h = torch.empty(((C_h.shape[-2] // 16) * (C_h.shape[-1] // 16),), dtype=torch.int32,
+                               pin_memory=True)
 
     def to_host(t):
         h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
@@ -606,7 +610,7 @@ def run_gpu(args):
 
     def e2e_step():
         if mode == "store":
-            return mmaemu.gemm_host(model, fmt, A_h, B_h, C_h, device=dev)
+            return mmaemu.gemm_host(model, fmt, A_h, B_h, C_h, device=dev, out=D_out_h, fp_out=fp_out_h)
         if spec["kind"] == "gemm":
             Ad, Bd, Cd = (t.to(dev, non_blocking=True) for t in (A_h, B_h, C_h))
             if mode == "fponly":

@@ -354,12 +354,16 @@ def xorsum(t) -> int:
     return int(res.value)
 
 
-def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bool = True, device=None):
+def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bool = True, device=None,
+              out=None, fp_out=None):
     """End-to-end call from host memory (mmaemu_gemm_host): host A, B (and C)
     in, host D and fingerprints out, with the transfers overlapped with the
     arithmetic inside the library.  Host tensors should be page-locked
     (``tensor.pin_memory()``) for the overlap.  ``device`` selects the CUDA
-    device (default: the current one).  Returns CPU tensors (D, fp)."""
+    device (default: the current one).  ``out`` / ``fp_out`` take the results
+    in caller-owned host tensors (contiguous, 32-bit elements: [M, N] and
+    [(M/16)*(N/16)]; fp_out implies fingerprint); otherwise page-locked
+    ones are allocated per call.  Returns CPU tensors (D, fp)."""
     torch = _torch()
     mi, fi = _model_fmt(model, fmt)
     for t, name in ((A_host, "A"), (B_host, "B")):
@@ -375,8 +379,21 @@ def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bo
         if C_host.is_cuda or not C_host.is_contiguous() or tuple(C_host.shape) != (M, N) or \
                 C_host.dtype not in (torch.float32, torch.int32, torch.uint32):
             raise TypeError("C must be a contiguous CPU fp32 tensor [M,N]")
-    D_host = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
-    fp_host = torch.empty(((M // 16) * (N // 16),), dtype=torch.int32, pin_memory=True) if fingerprint else None
+    words = (torch.float32, torch.int32, torch.uint32)
+    if out is not None:
+        if not isinstance(out, torch.Tensor) or out.is_cuda or not out.is_contiguous() or \
+                tuple(out.shape) != (M, N) or out.dtype not in words:
+            raise TypeError("out must be a contiguous CPU tensor [M,N] of 32-bit elements")
+        D_host = out
+    else:
+        D_host = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
+    if fp_out is not None:
+        if not isinstance(fp_out, torch.Tensor) or fp_out.is_cuda or not fp_out.is_contiguous() or \
+                fp_out.numel() != (M // 16) * (N // 16) or fp_out.dtype not in words[1:]:
+            raise TypeError("fp_out must be a contiguous CPU int32 tensor of (M/16)*(N/16) elements")
+        fp_host = fp_out
+    else:
+        fp_host = torch.empty(((M // 16) * (N // 16),), dtype=torch.int32, pin_memory=True) if fingerprint else None
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
         set_stream(torch.cuda.current_stream())
         fn = lib().mmaemu_gemm_host

@@ -175,3 +175,25 @@ def test_binding_refuses_operands_on_different_devices():
         mm._device_of(_FakeTensor("cuda:0"), _FakeTensor("cuda:1"))
     with pytest.raises(TypeError):
         mm._device_of(_FakeTensor("cpu"))
+
+
+def test_gemm_host_refuses_bad_output_buffers():
+    """gemm_host's caller-owned outputs are checked on the host, before the
+    library is called: D must be a contiguous CPU [M, N] tensor of 32-bit
+    elements, the fingerprints (M/16)*(N/16) 32-bit integers."""
+    import torch
+
+    import bit_exact_tensor_b200 as mm
+
+    M, N, K = 32, 48, 16
+    A = torch.zeros((M, K), dtype=torch.int16)
+    B = torch.zeros((K, N), dtype=torch.int16)
+    good_d = torch.zeros((M, N), dtype=torch.float32)
+    for bad in (torch.zeros((M, N + 16), dtype=torch.float32), torch.zeros((M, N), dtype=torch.float64),
+                torch.zeros((N, M), dtype=torch.float32).t()):
+        with pytest.raises(TypeError, match="out must be"):
+            mm.gemm_host("ampere", "fp16", A, B, None, out=bad)
+    for bad in (torch.zeros(((M // 16) * (N // 16) + 1,), dtype=torch.int32),
+                torch.zeros(((M // 16) * (N // 16),), dtype=torch.float32)):
+        with pytest.raises(TypeError, match="fp_out must be"):
+            mm.gemm_host("ampere", "fp16", A, B, None, out=good_d, fp_out=bad)

@@ -145,6 +145,15 @@ def test_gemm_from_host_memory(cref, shape, pinned):
     assert np.array_equal(fp.numpy().view(np.uint32), cref.tile_fingerprints(want))
     D0, _ = mmaemu.gemm_host("hopper", "fp16", host(A), host(B), None, fingerprint=False)
     assert np.array_equal(D0.view(torch.int32).numpy().view(np.uint32), cref.gemm("hopper", "fp16", A, B, None))
+    # into caller-owned host buffers (page-locked or not, as the inputs)
+    Dc = torch.full((M, N), -1, dtype=torch.int32)
+    fc = torch.full(((M // 16) * (N // 16),), -1, dtype=torch.int32)
+    if pinned:
+        Dc, fc = Dc.pin_memory(), fc.pin_memory()
+    D1, fp1 = mmaemu.gemm_host("ampere", "fp16", host(A), host(B), host(C), out=Dc, fp_out=fc)
+    assert D1 is Dc and fp1 is fc
+    assert np.array_equal(Dc.numpy().view(np.uint32), want)
+    assert np.array_equal(fc.numpy().view(np.uint32), cref.tile_fingerprints(want))
 
 
 def test_null_c_in_place_and_no_fingerprint(cref):

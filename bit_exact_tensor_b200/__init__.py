@@ -16,7 +16,7 @@ import os
 import threading
 
 __all__ = ["MODELS", "FORMATS", "MmaEmuError", "lib", "tiles", "gemm", "gemm_verify", "gemm_batched", "xorsum",
-           "xorsum_noalloc", "gemm_host", "set_stream", "trim_workspace", "set_workspace_cache", "workspace_reserved",
+           "xorsum_noalloc", "gemm_host", "tiles_host", "set_stream", "trim_workspace", "set_workspace_cache", "workspace_reserved",
            "device_status", "selftest_wait_timeout", "bounds_checking", "NO_MISMATCH"]
 
 MODELS = {"ampere": 0, "hopper": 1, "b200": 2, "lovelace": 0}
@@ -403,6 +403,44 @@ def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bo
                   C_host.data_ptr() if C_host is not None else None, D_host.data_ptr(),
                   fp_host.data_ptr() if fp_host is not None else None), "mmaemu_gemm_host")
     return D_host, fp_host
+
+
+def tiles_host(model: str, fmt: str, A_host, B_host, C_host=None, device=None, out=None):
+    """End-to-end tile batch from host memory (mmaemu_tiles_host): host A, B
+    (and C) [ntiles,16,16] in, host D out, streamed in chunks with the copies
+    in both directions overlapped with the arithmetic.  Host tensors should
+    be page-locked (``tensor.pin_memory()``).  ``out`` takes D in a
+    caller-owned contiguous CPU tensor of ntiles*256 32-bit elements;
+    otherwise a page-locked one is allocated.  Returns the CPU tensor D."""
+    torch = _torch()
+    mi, fi = _model_fmt(model, fmt)
+    for t, name in ((A_host, "A"), (B_host, "B")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CPU tensor")
+        if t.dtype not in _in_dtypes()[fmt]:
+            raise TypeError(f"{name} has dtype {t.dtype}, expected one of {_in_dtypes()[fmt]} for {fmt}")
+    nt = A_host.numel() // 256
+    if A_host.numel() != nt * 256 or B_host.numel() != nt * 256:
+        raise ValueError("A and B must hold ntiles x 16 x 16 elements each")
+    words = (torch.float32, torch.int32, torch.uint32)
+    if C_host is not None and (not isinstance(C_host, torch.Tensor) or C_host.is_cuda or
+                               not C_host.is_contiguous() or C_host.numel() != nt * 256 or C_host.dtype not in words):
+        raise TypeError("C must be a contiguous CPU fp32 tensor of ntiles x 16 x 16 elements")
+    if out is not None:
+        if not isinstance(out, torch.Tensor) or out.is_cuda or not out.is_contiguous() or \
+                out.numel() != nt * 256 or out.dtype not in words:
+            raise TypeError("out must be a contiguous CPU tensor of ntiles x 16 x 16 32-bit elements")
+        D_host = out
+    else:
+        D_host = torch.empty((nt, 16, 16), dtype=torch.float32, pin_memory=True)
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        set_stream(torch.cuda.current_stream())
+        fn = lib().mmaemu_tiles_host
+        fn.argtypes = [ctypes.c_int] * 2 + [ctypes.c_void_p] * 4 + [ctypes.c_size_t]
+        fn.restype = ctypes.c_int
+        _check(fn(mi, fi, A_host.data_ptr(), B_host.data_ptr(), C_host.data_ptr() if C_host is not None else None,
+                  D_host.data_ptr(), nt), "mmaemu_tiles_host")
+    return D_host
 
 
 def xorsum_noalloc(t) -> int:

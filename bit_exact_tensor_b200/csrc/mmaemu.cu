@@ -1742,6 +1742,89 @@ int launch_tiles(const void *A, const void *B, const float *C, float *D, size_t 
   return cudaGetLastError() == cudaSuccess ? MMAEMU_OK : MMAEMU_ECUDA;
 }
 
+// mmaemu_tiles from host memory: the tiles go in chunks.  A chunk's A, B
+// and C are copied in on a library copy stream, its tiles run on the
+// selected stream once they have arrived, and its D goes back on a second
+// copy stream, so that the copies in both directions overlap each other and
+// the arithmetic.
+constexpr int kTileHostMaxChunks = 8;
+constexpr size_t kTileHostMinChunk = 4096;  // tiles per chunk, at least (a chunk of fewer is one launch)
+template <int MODEL, int FMT>
+int launch_tiles_host(const void *A_h, const void *B_h, const float *C_h, float *D_h, size_t ntiles, int sms) {
+  constexpr size_t ES = FMT == mmaemu::FMT_E4M3 ? 1 : 2;
+  cudaStream_t s_in, s_out, c2;
+  int rc = host_streams(s_in, s_out, c2);
+  if (rc != MMAEMU_OK) return rc;
+  size_t nch = ntiles / kTileHostMinChunk;
+  nch = nch < 1 ? 1 : nch > (size_t)kTileHostMaxChunks ? (size_t)kTileHostMaxChunks : nch;
+  const size_t per = (ntiles + nch - 1) / nch;
+  nch = (ntiles + per - 1) / per;
+  const size_t ab_bytes = ntiles * 256 * ES, cd_bytes = ntiles * 256 * 4;
+  const size_t o_b = up256(ab_bytes), o_c = o_b + up256(ab_bytes), o_d = o_c + (C_h ? up256(cd_bytes) : 0);
+  const size_t total = o_d + up256(cd_bytes);
+  unsigned char *buf = nullptr;
+  cudaMemPool_t pool = workspace_pool();
+  if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void **>(&buf), total, pool, t_stream) != cudaSuccess)
+    return MMAEMU_ECUDA;
+  unsigned char *dA = buf, *dB = buf + o_b;
+  float *dC = C_h ? reinterpret_cast<float *>(buf + o_c) : nullptr;
+  float *dD = reinterpret_cast<float *>(buf + o_d);
+
+  const int nev = 2 + 2 * (int)nch;
+  cudaEvent_t ev[2 + 2 * kTileHostMaxChunks];
+  int made = 0;
+  for (; made < nev; made++)
+    if (cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming) != cudaSuccess) {
+      rc = MMAEMU_ECUDA;
+      break;
+    }
+  cudaEvent_t &e_alloc = ev[0], &e_out = ev[nev - 1];
+  auto e_in = [&](size_t ch) -> cudaEvent_t & { return ev[1 + ch]; };
+  auto e_done = [&](size_t ch) -> cudaEvent_t & { return ev[1 + nch + ch]; };
+  auto ok = [&](cudaError_t e) {
+    if (e != cudaSuccess) rc = MMAEMU_ECUDA;
+    return rc == MMAEMU_OK;
+  };
+  if (rc == MMAEMU_OK && ok(cudaEventRecord(e_alloc, t_stream)) && ok(cudaStreamWaitEvent(s_in, e_alloc, 0)))
+    ok(cudaStreamWaitEvent(s_out, e_alloc, 0));
+  for (size_t ch = 0; ch < nch && rc == MMAEMU_OK; ch++) {
+    const size_t t0 = ch * per, n = t0 + per < ntiles ? per : ntiles - t0;
+    const size_t ab0 = t0 * 256 * ES, abn = n * 256 * ES;
+    if (!ok(cudaMemcpyAsync(dA + ab0, static_cast<const unsigned char *>(A_h) + ab0, abn, cudaMemcpyHostToDevice,
+                            s_in)) ||
+        !ok(cudaMemcpyAsync(dB + ab0, static_cast<const unsigned char *>(B_h) + ab0, abn, cudaMemcpyHostToDevice,
+                            s_in)))
+      break;
+    if (C_h && !ok(cudaMemcpyAsync(dC + t0 * 256, C_h + t0 * 256, n * 256 * 4, cudaMemcpyHostToDevice, s_in)))
+      break;
+    ok(cudaEventRecord(e_in(ch), s_in));
+  }
+  for (size_t ch = 0; ch < nch && rc == MMAEMU_OK; ch++) {
+    const size_t t0 = ch * per, n = t0 + per < ntiles ? per : ntiles - t0;
+    if (!ok(cudaStreamWaitEvent(t_stream, e_in(ch), 0))) break;
+    rc = launch_tiles<MODEL, FMT>(dA + t0 * 256 * ES, dB + t0 * 256 * ES, dC ? dC + t0 * 256 : nullptr,
+                                  dD + t0 * 256, n, sms);
+    if (rc != MMAEMU_OK || !ok(cudaEventRecord(e_done(ch), t_stream)) ||
+        !ok(cudaStreamWaitEvent(s_out, e_done(ch), 0)))
+      break;
+    if (!ok(cudaMemcpyAsync(D_h + t0 * 256, dD + t0 * 256, n * 256 * 4, cudaMemcpyDeviceToHost, s_out))) break;
+  }
+  // the buffers go back to the pool once every copy has finished
+  if (made == nev) {
+    ok(cudaEventRecord(e_out, s_out));
+    ok(cudaStreamWaitEvent(t_stream, e_out, 0));
+    ok(cudaEventRecord(e_in(nch - 1), s_in));
+    ok(cudaStreamWaitEvent(t_stream, e_in(nch - 1), 0));
+  } else {
+    cudaStreamSynchronize(s_in);
+    cudaStreamSynchronize(s_out);
+  }
+  if (cudaFreeAsync(buf, t_stream) != cudaSuccess) rc = MMAEMU_ECUDA;
+  if (cudaStreamSynchronize(t_stream) != cudaSuccess) rc = MMAEMU_ECUDA;
+  for (int i = 0; i < made; i++) cudaEventDestroy(ev[i]);
+  return rc;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1763,6 +1846,19 @@ int mmaemu_tiles(int model, int fmt, const void *A, const void *B, const float *
 #define CALL_TILES(M_, F_) launch_tiles<M_, F_>(A, B, C, D, ntiles, sms)
   MMAEMU_DISPATCH(model, fmt, CALL_TILES);
 #undef CALL_TILES
+}
+
+int mmaemu_tiles_host(int model, int fmt, const void *A, const void *B, const float *C, float *D, size_t ntiles) {
+  if (!valid_pair(model, fmt)) return MMAEMU_EINVAL;
+  if (ntiles == 0) return MMAEMU_OK;
+  if (!A || !B || !D) return MMAEMU_EINVAL;
+  if (ntiles > ((size_t)1 << 40)) return MMAEMU_EINVAL;
+  int sms = 0;
+  const int rc = check_device(&sms);
+  if (rc != MMAEMU_OK) return rc;
+#define CALL_TILES_HOST(M_, F_) launch_tiles_host<M_, F_>(A, B, C, D, ntiles, sms)
+  MMAEMU_DISPATCH(model, fmt, CALL_TILES_HOST);
+#undef CALL_TILES_HOST
 }
 
 int mmaemu_native_tiles(int fmt, const void *A, const void *B, const float *C, float *D, size_t ntiles) {

@@ -181,6 +181,20 @@ int mmaemu_gemm_strided_batched(int model, int fmt, int trans_a, int trans_b, in
 int mmaemu_gemm_host(int model, int fmt, int M, int N, int K, const void *A, const void *B,
                      const float *C, float *D, uint32_t *fingerprint_out);
 
+/* mmaemu_tiles from and to HOST memory, synchronous: A, B, C (C may be NULL)
+ * and D are host pointers with the layouts of mmaemu_tiles (no alignment
+ * rule; D may equal C).  The tiles go in chunks of at least 4096 (at most 8
+ * chunks): a chunk's A, B and C are copied to the device on a library-owned
+ * copy stream, its tiles run on the selected stream once they have arrived,
+ * and its D is copied back on a second copy stream, so that the copies in
+ * both directions overlap each other and the arithmetic.  Page-locked host
+ * memory lets the copies run asynchronously.  Device memory comes from the
+ * library's workspace pool.  Returns after D is in host memory.
+ * ntiles == 0 is a no-op.  Errors: as mmaemu_tiles; MMAEMU_ECUDA also for a
+ * failed copy.                                                              */
+int mmaemu_tiles_host(int model, int fmt, const void *A, const void *B, const float *C, float *D,
+                      size_t ntiles);
+
 /* xorsum of n 32-bit words at device pointer D (the AEGIS fingerprint of a
  * whole tensor), written to *out_host.  SYNCHRONOUS: returns after the
  * result is on the host (it waits for the selected stream).  n == 0 gives 0.

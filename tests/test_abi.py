@@ -51,7 +51,8 @@ def test_header_declares_the_boundary():
                                     "mmaemu_probe_normalization", "mmaemu_probe_precision", "mmaemu_probe_subnormal",
                                     "mmaemu_probe_writeback_rounding", "mmaemu_selftest_wait_timeout",
                                     "mmaemu_set_stream", "mmaemu_set_workspace_cache", "mmaemu_strerror",
-                                    "mmaemu_tiles", "mmaemu_trim_workspace", "mmaemu_workspace_reserved",
+                                    "mmaemu_tiles", "mmaemu_tiles_host", "mmaemu_trim_workspace",
+                                    "mmaemu_workspace_reserved",
                                     "mmaemu_xorsum", "mmaemu_xorsum_noalloc"]
 
 
@@ -197,3 +198,21 @@ def test_gemm_host_refuses_bad_output_buffers():
                 torch.zeros(((M // 16) * (N // 16),), dtype=torch.float32)):
         with pytest.raises(TypeError, match="fp_out must be"):
             mm.gemm_host("ampere", "fp16", A, B, None, out=good_d, fp_out=bad)
+
+
+def test_tiles_host_refuses_bad_buffers():
+    """tiles_host checks its host tensors before the library is called."""
+    import torch
+
+    import bit_exact_tensor_b200 as mm
+
+    A = torch.zeros((3, 16, 16), dtype=torch.int16)
+    B = torch.zeros((3, 16, 16), dtype=torch.int16)
+    with pytest.raises(ValueError, match="ntiles"):
+        mm.tiles_host("ampere", "fp16", A, torch.zeros((2, 16, 16), dtype=torch.int16))
+    with pytest.raises(TypeError, match="A has dtype"):
+        mm.tiles_host("ampere", "fp16", A.float(), B)
+    with pytest.raises(TypeError, match="C must be"):
+        mm.tiles_host("ampere", "fp16", A, B, torch.zeros((3, 16, 16), dtype=torch.float64))
+    with pytest.raises(TypeError, match="out must be"):
+        mm.tiles_host("ampere", "fp16", A, B, None, out=torch.zeros((2, 16, 16), dtype=torch.float32))

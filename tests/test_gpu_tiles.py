@@ -111,3 +111,42 @@ def test_full_width_group_sums(cref, model, fmt):
     got = run_tiles(model, fmt, A, B, C)
     want = cref.tiles(model, fmt, A, B, C)
     assert np.array_equal(got, want), first_mismatch(got, want)
+
+
+def _host(x, pinned=True):
+    import torch
+
+    v = x.view(np.uint8) if x.dtype == np.uint8 else x.view(np.int16) if x.dtype == np.uint16 else x.view(np.int32)
+    t = torch.from_numpy(np.ascontiguousarray(v))
+    return t.pin_memory() if pinned else t
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_config2_from_host_memory(cref, pinned):
+    """mmaemu_tiles_host, the end-to-end tile call: 100,000 tiles streamed
+    in 8 chunks of 12,500 from host memory, the same bits as the oracle."""
+    import bit_exact_tensor_b200 as mmaemu
+
+    A, B, C, _ = wl.config2("fp16")
+    D = mmaemu.tiles_host("ampere", "fp16", _host(A, pinned), _host(B, pinned), _host(C, pinned))
+    got = D.view(-1).numpy().view(np.uint32).reshape(A.shape[0], 16, 16)
+    want = cref.tiles("ampere", "fp16", A, B, C)
+    assert np.array_equal(got, want), first_mismatch(got, want)
+
+
+@pytest.mark.parametrize("model,fmt,ntiles", [("hopper", "e4m3", 12305), ("ampere", "bf16", 4097), ("b200", "fp16", 1)])
+def test_ragged_chunks_from_host_memory(cref, model, fmt, ntiles):
+    """Chunk counts and ragged last chunks (12,305 tiles: three chunks of
+    4,102, 4,102 and 4,101; 4,097 tiles: one chunk), C = NULL, and D written
+    into a caller-owned buffer."""
+    import torch
+
+    import bit_exact_tensor_b200 as mmaemu
+
+    A, B, _ = wl.tiles_random_normal(ntiles, fmt, seed=ntiles, subnormal_frac=0.1)
+    out = torch.full((ntiles * 256,), -1, dtype=torch.int32).pin_memory()
+    D = mmaemu.tiles_host(model, fmt, _host(A), _host(B), None, out=out)
+    assert D is out
+    got = out.numpy().view(np.uint32).reshape(ntiles, 16, 16)
+    want = cref.tiles(model, fmt, A, B, None)
+    assert np.array_equal(got, want), first_mismatch(got, want)

@@ -990,7 +990,6 @@ __global__ void __launch_bounds__(GTHREADS, MMAEMU_GMINB) gemm_kernel(const Gemm
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row0 = rb * GBM, col0 = cb * GBN;
-  // this thread's 4 x 8 outputs
   // warp tiles of 32 x 64 outputs, lanes 4 x 8, 8 x 8 outputs each
   const int rl = warp * 32 + (lane >> 3) * GR;
   const int cl = (lane & 7) * GCC;

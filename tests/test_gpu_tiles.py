@@ -150,3 +150,18 @@ def test_ragged_chunks_from_host_memory(cref, model, fmt, ntiles):
     got = out.numpy().view(np.uint32).reshape(ntiles, 16, 16)
     want = cref.tiles(model, fmt, A, B, None)
     assert np.array_equal(got, want), first_mismatch(got, want)
+
+
+def test_tiles_from_host_memory_empty_and_invalid_pair():
+    """An empty batch is a no-op; an invalid model/format pair (Ampere has
+    no E4M3) is refused with MMAEMU_EINVAL before anything is copied."""
+    import torch
+
+    import bit_exact_tensor_b200 as mmaemu
+
+    empty = torch.zeros((0, 16, 16), dtype=torch.int16)
+    assert mmaemu.tiles_host("hopper", "fp16", empty, empty).numel() == 0
+    A = torch.zeros((2, 16, 16), dtype=torch.uint8)
+    with pytest.raises(mmaemu.MmaEmuError) as err:
+        mmaemu.tiles_host("ampere", "e4m3", A, A)
+    assert err.value.code == -1

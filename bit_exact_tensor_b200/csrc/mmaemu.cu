@@ -1728,12 +1728,20 @@ int launch_tiles(const void *A, const void *B, const float *C, float *D, size_t 
   auto kern = mmaemu::tiles_kernel<MODEL, FMT>;
   constexpr int TPB = 2 * mmaemu::T4WARPS;  // tiles per block and pass
   constexpr int THREADS = mmaemu::T4WARPS * 32;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return MMAEMU_ECUDA;
-  int per_sm = 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, smem) != cudaSuccess)
-    return MMAEMU_ECUDA;
-  if (per_sm < 1) per_sm = 1;
+  // the shared-memory attribute and the resident blocks per SM, once per
+  // device (a batch of tiles is short, so the per-call host time shows)
+  static std::atomic<int> s_per_sm[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MMAEMU_ECUDA;
+  int per_sm = s_per_sm[dev].load(std::memory_order_acquire);
+  if (per_sm == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return MMAEMU_ECUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, smem) != cudaSuccess)
+      return MMAEMU_ECUDA;
+    if (per_sm < 1) per_sm = 1;
+    s_per_sm[dev].store(per_sm, std::memory_order_release);
+  }
   const size_t want = (ntiles + TPB - 1) / TPB;
   const size_t cap = (size_t)sms * per_sm;
   const unsigned blocks = (unsigned)(want < cap ? want : cap);

@@ -442,6 +442,11 @@ def reduce_max(x: float, dist=None, device=None) -> float:
     return float(t.item())
 
 
+def any_rank(flag: bool, dist=None, device=None) -> bool:
+    """True on every rank when the flag is set on any rank."""
+    return reduce_max(1.0 if flag else 0.0, dist, device) > 0.0
+
+
 def aggregate_value(step_ms_max: float, world: int, macs_per_step: int = MACS_PER_STEP) -> float:
     """Whole-job emulated MACs/s: every rank runs one full problem per step
     (weak scaling), timed by the slowest rank."""
@@ -523,17 +528,17 @@ def run_gpu(args):
         def step():
             mmaemu.tiles(spec["model"], spec["fmt"], A, B, C, out=D)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-
     def timed():
-        """K steps between a barrier and a synchronisation, timed by events
-        around the whole run (the value), then K more with an event pair
-        around each call (each launch's duration, for the roofline).  The
-        first pass records nothing between steps: for the short tile batches
-        the per-step event records cost enough host time to leave the GPU
-        idle between calls."""
+        """W untimed warm-up steps right before the timed ones (the clock
+        sampler has just started and left the GPU idle), then K steps between
+        a barrier and a synchronisation, timed by events around the whole run
+        (the value), then K more with an event pair around each call (each
+        launch's duration, for the roofline).  The first timed pass records
+        nothing between steps: for the short tile batches the per-step event
+        records cost enough host time to leave the GPU idle between calls."""
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         barrier()
@@ -558,7 +563,9 @@ def run_gpu(args):
     with ClockSampler(local) as cs:
         total_ms, per_ms = timed()
     clocks = cs.summary()
-    if clocks_bad(clocks):
+    # re-measured on every rank when any rank's clock record is bad (the
+    # timed steps hold barriers, so all ranks take them together)
+    if any_rank(clocks_bad(clocks), dist, dev):
         with ClockSampler(local) as cs:
             total_ms, per_ms = timed()
         clocks = cs.summary()

@@ -107,3 +107,32 @@ def test_verify_full_size_e4m3():
     flat[0] ^= 1 << 20
     mism, _ = mmaemu.gemm_verify("hopper", "e4m3", Ad, Bd, None, D)
     assert mism.cpu().tolist() == [len(picks) - 1, picks[1]]
+
+
+@pytest.mark.parametrize("model,fmt", [("ampere", "fp16"), ("hopper", "bf16"), ("hopper", "e4m3")])
+def test_corrupted_input_byte_is_localised_by_the_fingerprints(cref, model, fmt):
+    """Fault injection on the host (the silent-data-corruption check the
+    fingerprints exist for): one exponent bit of one A element is flipped.
+    The recomputed per-tile fingerprints differ from the clean run's in that
+    element's row of tiles only, and equal the oracle's for the corrupted
+    input; one flipped bit in a host copy of D changes the whole-tensor
+    xorsum by exactly that bit."""
+    import bit_exact_tensor_b200 as mmaemu
+
+    M, N, K = 96, 160, 64
+    A, B, C = normal_inputs(M, N, K, fmt, seed=45)
+    D0, fp0 = mmaemu.gemm(model, fmt, dev_in(A), dev_in(B), dev_f32(C))
+    fp0 = host_bits(fp0).reshape(M // 16, N // 16)
+    m, k = 37, 21
+    bad = A.copy()
+    bad[m, k] ^= 0x40 if fmt == "e4m3" else 0x2000  # an exponent bit: the element's magnitude changes by 2^8 or more
+    _, fp1 = mmaemu.gemm(model, fmt, dev_in(bad), dev_in(B), dev_f32(C))
+    fp1 = host_bits(fp1).reshape(M // 16, N // 16)
+    assert np.array_equal(fp1.reshape(-1), cref.tile_fingerprints(cref.gemm(model, fmt, bad, B, C)))
+    rows = sorted(set(np.argwhere(fp1 != fp0)[:, 0].tolist()))
+    assert rows == [m // 16]
+    # one bit of D flipped on the host: the tensor's xorsum changes by that bit
+    d = host_bits(D0).reshape(-1).copy()
+    x0 = int(np.bitwise_xor.reduce(d))
+    d[1234] ^= np.uint32(1 << 17)
+    assert mmaemu.xorsum(dev_f32(d.reshape(M, N))) == x0 ^ (1 << 17)

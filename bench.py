@@ -65,7 +65,8 @@ GOLDEN = os.path.join(ROOT, "tests", "golden", "fullsize_gemm.json")
 GOLDEN_NAMES = {"gemm-ampere-fp16-4096": ("workloads", "cfg3-ampere-fp16-4096"),
                 "gemm-hopper-bf16-4096": ("workloads", "cfg4-hopper-bf16-4096"),
                 "gemm-hopper-bf16-4096-wide": ("workloads", "cfg4b-hopper-bf16-4096-wide"),
-                "gemm-hopper-e4m3-8192x4096x14336": ("workloads", "cfg5-hopper-e4m3-8192x4096x14336")}
+                "gemm-hopper-e4m3-8192x4096x14336": ("workloads", "cfg5-hopper-e4m3-8192x4096x14336"),
+                "gemm-b200-fp16-4096": ("workloads", "cfg3-b200-fp16-4096")}
 PEAK_OPS = {"dfma": 0, "dadd": 1, "add_min_s16x2": 2, "lop3": 3, "imad": 4, "iadd": 5, "popc_xor": 6, "prmt": 7,
             "imnmx": 8, "ffma": 9,
             # pairs on independent chains (rate in pairs): do two pipes work at the same time?

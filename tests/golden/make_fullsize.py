@@ -56,6 +56,9 @@ def workloads():
         "cfg4-hopper-bf16-4096": ("hopper", "bf16", wl.config4),
         "cfg4b-hopper-bf16-4096-wide": ("hopper", "bf16", lambda: wl.config4(wide=True)),
         "cfg5-hopper-e4m3-8192x4096x14336": ("hopper", "e4m3", wl.config5),
+        # B200's own FP16 MMA as measured with the pages' target tests: the
+        # 4096^3 inputs of config 3 under that model
+        "cfg3-b200-fp16-4096": ("b200", "fp16", wl.config3),
     }
 
 

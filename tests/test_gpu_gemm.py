@@ -2,7 +2,8 @@
 
 Small and ragged shapes are compared element by element in full.  The
 full-size workloads (4096^3 FP16-Ampere, 4096^3 BF16-Hopper with and without
-out-of-range sums, 8192x4096x14336 E4M3-Hopper) run in the same launch
+out-of-range sums, 8192x4096x14336 E4M3-Hopper, and 4096^3 FP16 under the
+measured B200 model) run in the same launch
 configuration the benchmark times and are compared in full with the oracle's
 result through digests that tests/golden/make_fullsize.py stored from a run of
 the oracle on every output element: the SHA-256 of D (every element), the
@@ -206,6 +207,7 @@ FULL = {
     "cfg4-hopper-bf16-4096": ("hopper", "bf16", lambda: wl.config4()),
     "cfg4b-hopper-bf16-4096-wide": ("hopper", "bf16", lambda: wl.config4(wide=True)),
     "cfg5-hopper-e4m3-8192x4096x14336": ("hopper", "e4m3", lambda: wl.config5()),
+    "cfg3-b200-fp16-4096": ("b200", "fp16", lambda: wl.config3()),
 }
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "fullsize_gemm.json")
 

@@ -92,6 +92,7 @@ E4M3_LAYER = "gemm-hopper-e4m3-8192x4096x14336"
 # a claimed D instead of storing it, weights stored [N][K] (B transposed)
 GEMM_MODES = ("fponly", "verify", "wt")
 BATCHED = "gemm-batched-ampere-fp16-8x1024x4096x4096"
+GOLDEN_NAMES[BATCHED] = ("workloads", "batched-ampere-fp16-8x1024x4096x4096")
 WORKLOAD_NAMES = ({DEFAULT_WORKLOAD, "gemm-hopper-bf16-4096", "gemm-hopper-bf16-4096-wide", E4M3_LAYER,
                    "tiles-ampere-fp16-4096", BATCHED, "gemm-b200-fp16-4096"}
                   | {f"{E4M3_LAYER}-{m}" for m in GEMM_MODES}
@@ -586,7 +587,7 @@ def run_gpu(args):
         # and the claim itself (computed by the library) against the oracle's D
         verified = verify_against_oracle(args.workload.rsplit("-verify", 1)[0], D.cpu().numpy(), None)
         verified["against"] += "; the timed verify calls found 0 mismatches in that claim"
-    elif mode in ("store", "wt", None) or spec["kind"] == "tiles":
+    elif mode in ("store", "wt", "batched", None) or spec["kind"] == "tiles":
         # the last timed call's result against the oracle's stored digests
         # (only the plain GEMM call writes fingerprints here)
         base = args.workload[:-3] if mode == "wt" else args.workload  # B stored [N][K]: the same GEMM
@@ -672,7 +673,7 @@ def run_gpu(args):
         else:
             base = args.workload[:-3] if mode == "wt" else args.workload
             e2e_verified = verify_against_oracle(
-                base, Dh.numpy(), fph.numpy() if spec["kind"] == "gemm" and mode == "store" and fph is not None
+                base, Dh.numpy(), fph.numpy() if spec["kind"] == "gemm" and mode in ("store", "batched") and fph is not None
                 else None)["verified"]
 
     if rank == 0:

@@ -59,6 +59,9 @@ def workloads():
         # B200's own FP16 MMA as measured with the pages' target tests: the
         # 4096^3 inputs of config 3 under that model
         "cfg3-b200-fp16-4096": ("b200", "fp16", wl.config3),
+        # 8 independent 1024 x 4096 x 4096 problems (the layouts' batched
+        # GEMM): D stacked as [8 * 1024, 4096], fingerprints batch-major
+        "batched-ampere-fp16-8x1024x4096x4096": ("ampere", "fp16", lambda: wl.config_batched(8, 1024, 4096, 4096)),
     }
 
 
@@ -91,15 +94,24 @@ def run_one(name: str, threads: int) -> dict:
 
     model, fmt, make = workloads()[name]
     A, B, C = make()
-    M, K = A.shape
-    N = B.shape[1]
     t0 = time.perf_counter()
-    D = cref.gemm(model, fmt, A, B, C, nthreads=threads)
+    if A.ndim == 3:  # a batch of independent problems, one oracle run each
+        parts = [cref.gemm(model, fmt, A[b], B[b], C[b], nthreads=threads) for b in range(A.shape[0])]
+        fp = np.concatenate([cref.tile_fingerprints(Db) for Db in parts])
+        D = np.concatenate(parts, axis=0)
+        batch = A.shape[0]
+    else:
+        D = cref.gemm(model, fmt, A, B, C, nthreads=threads)
+        fp = cref.tile_fingerprints(D)
+        batch = 1
     dt = time.perf_counter() - t0
-    fp = cref.tile_fingerprints(D)
+    M, K = A.shape[-2:]
+    N = B.shape[-1]
     rec = {"model": model, "fmt": fmt, "M": M, "N": N, "K": K, "xorsum": cref.xorsum(D),
            "specials": special_counts(D), "oracle_seconds": round(dt, 2), "oracle_threads": threads,
-           "oracle_macs_per_s": M * N * K / dt}
+           "oracle_macs_per_s": batch * M * N * K / dt}
+    if batch > 1:
+        rec["batch"] = batch
     rec.update(digests(D, fp))
     return rec
 

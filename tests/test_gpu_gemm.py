@@ -260,6 +260,20 @@ def test_full_size_from_host_memory_equals_the_oracle(name):
     assert got["fp_sha256"] == rec["fp_sha256"], "tile fingerprints from host memory differ from the oracle's"
 
 
+def test_full_size_batched_equals_the_oracle():
+    """The batched workload (8 independent 1024 x 4096 x 4096 FP16-Ampere
+    problems in one strided-batched call) against the oracle's digests of the
+    stacked D and the batch-major tile fingerprints."""
+    import bit_exact_tensor_b200 as mmaemu
+
+    rec = golden_record("batched-ampere-fp16-8x1024x4096x4096")
+    A, B, C = wl.config_batched(8, 1024, 4096, 4096)
+    D, fp = mmaemu.gemm_batched("ampere", "fp16", dev_in(A), dev_in(B), dev_f32(C))
+    got = fullsize_digests(host_bits(D).reshape(-1, 4096), host_bits(fp))
+    assert got["d_sha256"] == rec["d_sha256"], "batched D differs from the oracle's"
+    assert got["fp_sha256"] == rec["fp_sha256"], "batched fingerprints differ from the oracle's"
+
+
 def test_full_size_deterministic():
     A, B, C = wl.config3()
     _, fp1 = run_gemm("ampere", "fp16", A, B, C)

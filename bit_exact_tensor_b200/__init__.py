@@ -355,7 +355,7 @@ def xorsum(t) -> int:
 
 
 def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bool = True, device=None,
-              out=None, fp_out=None):
+              out=None, fp_out=None, store_d: bool = True):
     """End-to-end call from host memory (mmaemu_gemm_host): host A, B (and C)
     in, host D and fingerprints out, with the transfers overlapped with the
     arithmetic inside the library.  Host tensors should be page-locked
@@ -363,7 +363,9 @@ def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bo
     device (default: the current one).  ``out`` / ``fp_out`` take the results
     in caller-owned host tensors (contiguous, 32-bit elements: [M, N] and
     [(M/16)*(N/16)]; fp_out implies fingerprint); otherwise page-locked
-    ones are allocated per call.  Returns CPU tensors (D, fp)."""
+    ones are allocated per call.  store_d=False is the fingerprint-only
+    mode: D is neither written nor copied back (None).  Returns CPU tensors
+    (D, fp)."""
     torch = _torch()
     mi, fi = _model_fmt(model, fmt)
     for t, name in ((A_host, "A"), (B_host, "B")):
@@ -380,7 +382,13 @@ def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bo
                 C_host.dtype not in (torch.float32, torch.int32, torch.uint32):
             raise TypeError("C must be a contiguous CPU fp32 tensor [M,N]")
     words = (torch.float32, torch.int32, torch.uint32)
-    if out is not None:
+    if not store_d:
+        if not fingerprint and fp_out is None:
+            raise ValueError("store_d=False needs fingerprint=True")
+        if out is not None:
+            raise ValueError("store_d=False writes no D: out must be None")
+        D_host = None
+    elif out is not None:
         if not isinstance(out, torch.Tensor) or out.is_cuda or not out.is_contiguous() or \
                 tuple(out.shape) != (M, N) or out.dtype not in words:
             raise TypeError("out must be a contiguous CPU tensor [M,N] of 32-bit elements")
@@ -400,7 +408,8 @@ def gemm_host(model: str, fmt: str, A_host, B_host, C_host=None, fingerprint: bo
         fn.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 5
         fn.restype = ctypes.c_int
         _check(fn(mi, fi, M, N, K, A_host.data_ptr(), B_host.data_ptr(),
-                  C_host.data_ptr() if C_host is not None else None, D_host.data_ptr(),
+                  C_host.data_ptr() if C_host is not None else None,
+                  D_host.data_ptr() if D_host is not None else None,
                   fp_host.data_ptr() if fp_host is not None else None), "mmaemu_gemm_host")
     return D_host, fp_host
 

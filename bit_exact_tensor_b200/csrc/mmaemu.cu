@@ -1588,7 +1588,8 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
   // device buffers, each 256-byte aligned inside one pool allocation; two
   // A-blob workspaces, one per compute stream
   const size_t o_b = up256(a_bytes), o_c = o_b + up256(b_bytes), o_d = o_c + (C_h ? up256(cd_bytes) : 0);
-  const size_t o_fp = o_d + up256(cd_bytes), o_wa = o_fp + up256(fp_bytes), o_wb = o_wa + 2 * up256(zs.a_bytes);
+  const size_t o_fp = o_d + (D_h ? up256(cd_bytes) : 0), o_wa = o_fp + up256(fp_bytes);
+  const size_t o_wb = o_wa + 2 * up256(zs.a_bytes);
   const size_t total = o_wb + up256(zb.b_bytes);
   unsigned char *buf = nullptr;
   cudaMemPool_t pool = workspace_pool();
@@ -1596,7 +1597,7 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
     return MMAEMU_ECUDA;
   unsigned char *dA = buf, *dB = buf + o_b;
   float *dC = C_h ? reinterpret_cast<float *>(buf + o_c) : nullptr;
-  float *dD = reinterpret_cast<float *>(buf + o_d);
+  float *dD = D_h ? reinterpret_cast<float *>(buf + o_d) : nullptr;  // fingerprint-only: no D at all
   uint32_t *dfp = fp_h ? reinterpret_cast<uint32_t *>(buf + o_fp) : nullptr;
 
   const int nev = 2 + 2 * nslab + 3;
@@ -1641,7 +1642,7 @@ int launch_gemm_host(int M, int N, int K, const void *A_h, const void *B_h, cons
     q.M = rows;
     q.A = dA + r0 * K * ES;
     q.C = dC ? dC + r0 * N : nullptr;
-    q.D = dD + r0 * N;
+    q.D = dD ? dD + r0 * N : nullptr;
     q.fp = dfp ? dfp + (r0 / 16) * (N / 16) : nullptr;
     q.dA = buf + o_wa + (sl & 1) * up256(zs.a_bytes);
     q.dA_n = zs.a_bytes;

@@ -155,6 +155,10 @@ def test_gemm_from_host_memory(cref, shape, pinned):
     assert D1 is Dc and fp1 is fc
     assert np.array_equal(Dc.numpy().view(np.uint32), want)
     assert np.array_equal(fc.numpy().view(np.uint32), cref.tile_fingerprints(want))
+    # fingerprints only: no D on the device or in host memory
+    D2, fp2 = mmaemu.gemm_host("ampere", "fp16", host(A), host(B), host(C), store_d=False)
+    assert D2 is None
+    assert np.array_equal(fp2.numpy().view(np.uint32), cref.tile_fingerprints(want))
 
 
 def test_null_c_in_place_and_no_fingerprint(cref):

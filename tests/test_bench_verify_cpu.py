@@ -44,3 +44,24 @@ def test_one_flipped_bit_is_rejected(bench_mod, oracle_d):
 def test_unknown_workload_is_not_claimed_verified(bench_mod, oracle_d):
     rec = bench_mod.verify_against_oracle("no-such-workload", oracle_d.view(np.float32), None)
     assert rec["verified"] is None
+
+
+def test_every_benchmark_workload_has_stored_oracle_digests(bench_mod):
+    """Each workload bench.py can time (its modes -fponly, -verify and -wt
+    share their base workload's result) maps to a record of oracle digests,
+    so no timed result goes unchecked."""
+    import json
+
+    with open(bench_mod.GOLDEN) as fh:
+        golden = json.load(fh)
+    for name in sorted(bench_mod.WORKLOAD_NAMES):
+        base = name
+        for suffix in ("-fponly", "-verify", "-wt"):
+            if base.endswith(suffix):
+                base = base[: -len(suffix)]
+        assert base in bench_mod.GOLDEN_NAMES, name
+        sec, key = bench_mod.GOLDEN_NAMES[base]
+        rec = golden[sec][key]
+        assert len(rec["d_sha256"]) == 64, name
+        if sec == "workloads":
+            assert len(rec["fp_sha256"]) == 64, name

@@ -8,7 +8,9 @@ access skipped (no trap, no fault).  A child process loads that build
 (MMAEMU_LIB=check), runs GEMMs of every layout and mode and tile batches on
 small and ragged shapes, compares them with the oracle, and requires the
 status word to stay clear -- a substitute for a memory checker, which this
-pool does not run.
+pool does not run.  A second child runs the full-size workloads (device and
+host-memory GEMMs, the batched GEMM, streamed tiles) against the oracle's
+stored digests under the same build.
 """
 
 import os
@@ -76,3 +78,54 @@ def test_checking_build_runs_clean_and_exact():
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=1200)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
     assert "CHECKED 21" in r.stdout
+
+
+FULL_CHILD = r"""
+import sys, json, hashlib
+sys.path.insert(0, ROOT); sys.path.insert(0, HERE)
+import numpy as np, torch
+import bit_exact_tensor_b200 as mmaemu
+from bit_exact_tensor_b200 import workloads as wl
+
+assert mmaemu.bounds_checking(), "not the checking build"
+mmaemu.device_status(clear=True)
+G = json.load(open(GOLDEN))
+sha = lambda x: hashlib.sha256(np.ascontiguousarray(x, dtype="<u4").tobytes()).hexdigest()
+
+def host(x):
+    v = x.view(np.uint8) if x.dtype == np.uint8 else x.view(np.int16) if x.dtype == np.uint16 else x.view(np.int32)
+    return torch.from_numpy(np.ascontiguousarray(v)).pin_memory()
+
+A, B, C = wl.config3()
+rec = G["workloads"]["cfg3-ampere-fp16-4096"]
+D, fp = mmaemu.gemm("ampere", "fp16", host(A).cuda(), host(B).cuda(), host(C).cuda())
+assert sha(D.cpu().numpy().view(np.uint32)) == rec["d_sha256"] and sha(fp.cpu().numpy().view(np.uint32)) == rec["fp_sha256"]
+Dh, fph = mmaemu.gemm_host("ampere", "fp16", host(A), host(B), host(C))
+assert sha(Dh.numpy().view(np.uint32)) == rec["d_sha256"] and sha(fph.numpy().view(np.uint32)) == rec["fp_sha256"]
+A, B, C = wl.config_batched(8, 1024, 4096, 4096)
+rec = G["workloads"]["batched-ampere-fp16-8x1024x4096x4096"]
+D, fp = mmaemu.gemm_batched("ampere", "fp16", host(A).cuda(), host(B).cuda(), host(C).cuda())
+assert sha(D.cpu().numpy().view(np.uint32).reshape(-1, 4096)) == rec["d_sha256"]
+assert sha(fp.cpu().numpy().view(np.uint32)) == rec["fp_sha256"]
+A, B, C, _ = wl.config2("fp16")
+Dt = mmaemu.tiles_host("ampere", "fp16", host(A), host(B), host(C))
+assert sha(Dt.numpy().view(np.uint32)) == G["tiles"]["tiles-ampere-fp16-100k"]["d_sha256"]
+torch.cuda.synchronize()
+bits = mmaemu.device_status()
+assert bits == 0, f"status word {bits:#x}"
+print("FULL CHECKED")
+"""
+
+
+def test_checking_build_at_full_size():
+    """The same build on the full-size workloads: the 4096^3 FP16-Ampere GEMM
+    from device and from host memory (row slabs on two compute streams), the
+    batched GEMM and 100,000 tiles streamed from host memory in chunks.  Every
+    result equals the oracle's stored digests and no index leaves its
+    buffer."""
+    env = dict(os.environ, MMAEMU_LIB="check")
+    golden = os.path.join(HERE, "golden", "fullsize_gemm.json")
+    code = "ROOT = %r\nHERE = %r\nGOLDEN = %r\n" % (ROOT, HERE, golden) + FULL_CHILD
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=1200)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert "FULL CHECKED" in r.stdout
